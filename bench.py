@@ -1,0 +1,344 @@
+"""Benchmark of the rolling-window attention layer hot path on B200.
+
+One step = one pass of the layer's hot path on the paper-shaped denoise
+workload: fused 3D-RoPE attention of 23,400 query tokens over 32,760 context
+tokens (12 heads, d = 128, bf16; RoPE on Q and K inside the kernel) plus the
+per-layer ring KV-cache update that inserts 5 frames (30x52 tokens, 12 heads)
+into a 21-slot ring.  Inputs are seeded N(0,1) bf16 draws resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Under torchrun with N > 1 every rank runs an
+independent replica of the same step (the path has no exchange step), the
+timed region is bracketed by a barrier + synchronize and the max over ranks is
+reported.  ``--impl reference`` times the CPU oracle on this host instead.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused-RoPE attention TFLOP/s @23.4k×32.8k (% bf16 peak); KV update GB/s"
+H, D = 12, 128
+GRID_H, GRID_W = 30, 52
+F = GRID_H * GRID_W
+LQ, LK = 15 * F, 21 * F
+Q_T0, K_T0 = 6, 0
+RING_SLOTS, RING_INSERT = 21, 5
+ATTN_FLOPS = 4.0 * LQ * LK * D * H                 # QK^T and PV, visible pairs only (no mask)
+RING_BYTES = 2 * 2 * RING_INSERT * F * H * D * 2    # (K and V) x (read + write)
+SEED = 1002
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def workload_config(n_gpus):
+    return {
+        "workload": "denoise_30x52_h12_q23400_k32760 + ring_21x1560x12_insert5",
+        "Lq": LQ, "Lk": LK, "heads": H, "head_dim": D, "frame_grid": [GRID_H, GRID_W],
+        "rope": "3D t/h/w pairs 22/21/21 theta 1e4, fused on Q and K",
+        "mask": "none", "ring": {"slots": RING_SLOTS, "insert_frames": RING_INSERT},
+        "global_batch": n_gpus, "seq_len": LQ, "parallelism": f"replicas x{n_gpus}",
+        "l2": "no flush: each step reads 273 MB of attention operands and moves 96 MB in the ring update, "
+              "both above the 126 MB L2",
+    }
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"bf16": j.get("bf16_tflops", 1590.0), "bf16_sustained": j.get("bf16_tflops_sustained", 1400.0),
+                "hbm": j.get("hbm_gbs", 6650.0), "source": "measured"}
+    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_inputs(device):
+    import torch
+    from rolling_kv_cache_rope_b200.synth import bf16_normal_bits
+
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+
+    qb = bf16_normal_bits(SEED, (LQ, H, D))
+    kb = bf16_normal_bits(SEED + 100, (LK, H, D))
+    vb = bf16_normal_bits(SEED + 200, (LK, H, D))
+    knb = bf16_normal_bits(SEED + 300, (RING_INSERT * F, H, D))
+    vnb = bf16_normal_bits(SEED + 400, (RING_INSERT * F, H, D))
+    host = {"q": qb, "k": kb, "v": vb, "k_new": knb, "v_new": vnb}
+    devt = {k: dev(v) for k, v in host.items()}
+    return host, devt
+
+
+def cpu_baseline(host, rows=256):
+    """Time the float64 oracle on a bounded sample: RoPE of all 32,760 keys and
+    of ``rows`` query rows, then attention for those rows (all 12 heads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    rows_idx = np.linspace(0, LQ - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.fused_attention_ref(oracle.bf16_bits_to_f64(host["q"]), oracle.bf16_bits_to_f64(host["k"]),
+                               oracle.bf16_bits_to_f64(host["v"]), scale=1 / math.sqrt(D), grid_h=GRID_H,
+                               grid_w=GRID_W, rope_q=True, rope_k=True, q_t0=Q_T0, k_t0=K_T0, rows=rows_idx)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * rows * LK * D * H
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"{rows} of {LQ} query rows x {H} heads over all {LK} keys, incl. fp64 RoPE of all keys; "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as it stands, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from rolling_kv_cache_rope_b200.synth import bf16_normal_bits
+    host = {"q": bf16_normal_bits(SEED, (LQ, H, D)), "k": bf16_normal_bits(SEED + 100, (LK, H, D)),
+            "v": bf16_normal_bits(SEED + 200, (LK, H, D))}
+    rows = 16
+    for _ in range(args.warmup):
+        cpu_baseline(host, rows)
+    t0 = time.perf_counter()
+    vals = [cpu_baseline(host, rows) for _ in range(args.steps)]
+    dt = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.gpus), "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from rolling_kv_cache_rope_b200 import rkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device, timeout=__import__("datetime").timedelta(seconds=120))
+
+    host, t = make_inputs(device)
+    rope = rkv.make_rope(GRID_H, GRID_W)
+    o = torch.empty((LQ, H, D), dtype=torch.bfloat16, device=device)
+    ring = rkv.KVRing(RING_SLOTS, F, H, D, device=device)
+    ws = torch.zeros(rkv.attn_fwd_varlen_workspace_size(1, H, D), dtype=torch.uint8, device=device)
+    seq = rkv.AttnSeq(t["q"], t["k"], t["v"], o, q_t0=Q_T0, k_t0=K_T0)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rkv.attn_fwd_varlen([seq], rope, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        rkv.kvcache_ring_update(ring, t["k_new"], t["v_new"], RING_INSERT)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    rkv.rkv_attn_status(ws)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    rkv.rkv_attn_status(ws)
+    total_ms = start.elapsed_time(end)
+    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    ring_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the two calls, D2H of the attention output
+    pinned = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in host.items()}
+    o_host = torch.empty((LQ, H, D), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for k in ("q", "k", "v", "k_new", "v_new"):
+            t[k].copy_(pinned[k], non_blocking=True)
+        rkv.attn_fwd_varlen([seq], rope, workspace=ws)
+        rkv.kvcache_ring_update(ring, t["k_new"], t["v_new"], RING_INSERT)
+        o_host.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+    h2d = sum(v.nbytes for v in host.values())
+    d2h = LQ * H * D * 2
+
+    if rank == 0:
+        peaks = measured_peaks()
+        ms_per_step = total_ms / args.steps
+        value = world * ATTN_FLOPS / (ms_per_step * 1e-3) / 1e12
+        attn_avg = statistics.mean(attn_ms)
+        ring_avg = statistics.mean(ring_ms)
+        achieved = ATTN_FLOPS / (attn_avg * 1e-3) / 1e12
+        traffic = load_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
+                         "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                         "frac_of_burst": achieved / peaks["bf16"],
+                         "frac_of_nominal_2250": achieved / NOMINAL_BF16_TFLOPS,
+                         "kernel": "attn_fwd_kernel", "avg_ms": attn_avg},
+            "kv_update": {"value": RING_BYTES / (ring_avg * 1e-3) / 1e9, "unit": "GB/s", "avg_us": ring_avg * 1e3,
+                          "bytes_per_call": RING_BYTES, "frac_of_measured_hbm": RING_BYTES / (ring_avg * 1e-3) / 1e9 / peaks["hbm"],
+                          "frac_of_nominal_8000": RING_BYTES / (ring_avg * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+            "e2e": {"value": world * ATTN_FLOPS * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(host)
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if the
+    kernel has not changed since it was captured (else null)."""
+    p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

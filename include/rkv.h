@@ -1,0 +1,233 @@
+/*
+ * rkv.h -- C ABI of librkv.so: rolling KV cache + fused 3D-RoPE attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Three operations make up the per-layer hot path of a streaming
+ * autoregressive-diffusion video model (Rolling Forcing as the proxy):
+ *
+ *   rope3d_apply         3D rotary embedding over (t, h, w) of Q or K
+ *   attn_fwd_varlen      softmax attention, RoPE fused into its load stage,
+ *                        several sequences (e.g. the denoise pass and the
+ *                        cache-update pass) in one launch, optional
+ *                        frame-block-causal mask
+ *   kvcache_ring_update  insert whole frames into a per-layer ring cache,
+ *                        evicting the oldest frames
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are bfloat16, token-major [L][H][D] ("row" = one token, H heads
+ *    of D = 128 values).  A row stride (in ELEMENTS) lets a caller pass a view
+ *    into a wider buffer (e.g. the Q part of a fused QKV projection); it must
+ *    be >= H*D and make every row start 16-byte aligned.  No call transposes.
+ *  - Pointers named device are CUDA device (or managed) memory; the caller owns
+ *    all of it.  The library allocates no device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls enqueue work and return without synchronising.
+ *  - Every call returns an rkv_status.  Invalid arguments are rejected on the
+ *    host BEFORE anything is launched; nothing traps or asserts on the device.
+ *    rkv_last_error_string() describes the last failure of the calling thread.
+ *  - Functions keep no global state between calls (the ring state lives in the
+ *    caller's rkv_ring).
+ */
+#ifndef RKV_H
+#define RKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RKV_OK = 0,
+  RKV_ERR_INVALID_ARG = 1, /* rejected on the host, nothing launched           */
+  RKV_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels handle  */
+  RKV_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed                */
+  RKV_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see below)   */
+} rkv_status;
+
+/*
+ * 3D-RoPE parameters.
+ *
+ * Source: "Amazon and Reactor tune Trainium for real-time video generation",
+ * section "Three problems for generic compilers": in video, RoPE rotates by
+ * three positions -- height, width and time -- instead of one.  The pages give
+ * no formula; this library takes the plainest reading:
+ *   token i of a sequence whose first frame has time index t0, on a
+ *   grid_h x grid_w frame grid (F = grid_h*grid_w tokens per frame, row-major):
+ *       t = t0 + i / F,  h = (i % F) / grid_w,  w = i % grid_w
+ *   the D/2 rotary pairs are adjacent elements (2j, 2j+1); the first pairs_t
+ *   pairs use t, the next pairs_h use h, the last pairs_w use w
+ *   (pairs_t + pairs_h + pairs_w == D/2; 22/21/21 for D = 128);
+ *   pair with local index k on an axis with n pairs turns by
+ *       angle = pos * theta^(-k/n)
+ *   y0 = x0 cos(angle) - x1 sin(angle);  y1 = x0 sin(angle) + x1 cos(angle).
+ */
+typedef struct {
+  int32_t grid_h, grid_w;            /* frame grid; tokens per frame = grid_h*grid_w */
+  int32_t pairs_t, pairs_h, pairs_w; /* rotary pairs per axis, sum = D/2            */
+  float theta;                       /* frequency base, 10000 for all three axes    */
+} rkv_rope3d;
+
+/*
+ * rope3d_apply -- y = RoPE3D(x) for every row and head.
+ *
+ * Source: "Optimizing Real-Time Video Generation on Trainium Chips", item 6
+ * "Neuron Kernel Interface" (a dedicated 3D-RoPE kernel replaced the generic
+ * path) and the RoPE reading above.
+ *
+ *   x, y          device bf16 [L][H][D]; y may equal x (in place), otherwise
+ *                 the two must not overlap.
+ *   L             rows (tokens), >= 0 (0 = no-op).  H >= 1.  D == 128.
+ *   x_row_stride, y_row_stride   elements between consecutive rows.
+ *   t0            time index of row 0's frame.
+ *   rope          frame grid and axis split.
+ * Precision: rotation in fp32 with a compensated (error-free-transform) path
+ * and fp64-derived cos/sin, rounded to nearest-even bf16: every output is
+ * within 1 bf16 ulp of the exactly rounded result.
+ * Errors: RKV_ERR_INVALID_ARG for null pointers, D != 128, bad pairs/grid,
+ * misaligned rows or overlapping non-identical x/y.
+ */
+rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H, int32_t D,
+                        int64_t x_row_stride, int64_t y_row_stride, int32_t t0,
+                        const rkv_rope3d* rope, void* stream);
+
+/* flags of rkv_attn_seq */
+#define RKV_ROPE_Q 1u /* rotate Q rows by RoPE3D (positions from q_t0) in-kernel */
+#define RKV_ROPE_K 2u /* rotate K rows by RoPE3D (positions from k_t0) in-kernel */
+
+/*
+ * One sequence of a batched attention launch.
+ *
+ * Source: SDPA of a 23,400-token query window over a 32,760-token context,
+ * 12 heads ("A kernel-centric path to real-time video generation on
+ * Trainium", ai4snews summary, second paragraph); two passes per window --
+ * denoise, then cache update -- with different attention lengths, batched so
+ * the lighter pass does not strand hardware ("Optimizing Real-Time Video
+ * Generation on Trainium Chips", item 8 "Model structure optimizations";
+ * "Amazon and Reactor tune Trainium for real-time video generation", section
+ * "Three problems for generic compilers").
+ *
+ *   q, k, v       device bf16 [Lq][H][D], [Lk][H][D], [Lk][H][D]
+ *   o             device bf16 [Lq][H][D]; must not overlap q, k or v
+ *   *_stride      elements between consecutive rows (>= H*D, 16-B aligned rows)
+ *   Lq, Lk        >= 1 each
+ *   q_t0, k_t0    time index of the first query / key frame (used for RoPE)
+ *   block_frames  0 = every key visible.  > 0 = frame-block causal: query row r
+ *                 lies in key frame qf = q_frame_offset + r / F, key c in key
+ *                 frame c / F, and key c is visible iff
+ *                 floor(kf / block_frames) <= floor(qf / block_frames).
+ *                 (F = tokens per frame from rkv_rope3d.)
+ *   q_frame_offset key-frame index of query frame 0 (>= 0); the bottom-right
+ *                 alignment (query window = last frames of the context) is
+ *                 Lk/F - Lq/F.
+ *   flags         RKV_ROPE_Q | RKV_ROPE_K
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  int64_t q_stride, k_stride, v_stride, o_stride;
+  int32_t Lq, Lk;
+  int32_t q_t0, k_t0;
+  int32_t q_frame_offset;
+  int32_t block_frames;
+  uint32_t flags;
+  int32_t reserved; /* must be 0 */
+} rkv_attn_seq;
+
+#define RKV_MAX_SEQS 16
+
+/*
+ * attn_fwd_varlen -- O = softmax(mask(RoPE(Q) RoPE(K)^T * softmax_scale)) V
+ * for every sequence and head, in ONE kernel launch.
+ *
+ *   seqs, n_seqs   host array of 1..RKV_MAX_SEQS descriptors (read during the
+ *                  call only)
+ *   H >= 1, D == 128, softmax_scale > 0 (1/sqrt(128) for SDPA)
+ *   rope           frame grid / axis split; required (also defines F for the
+ *                  mask) even when no sequence sets a RoPE flag
+ *   workspace      device memory of at least attn_fwd_varlen_workspace_size()
+ *                  bytes, 16-byte aligned, not used by another call in flight;
+ *                  holds the device status word.  May be NULL only when that
+ *                  size is 0.
+ * A query row that sees no key gets zeros.  Precision: bf16 operands, fp32
+ * accumulation and softmax, bf16 output.
+ * Errors: RKV_ERR_INVALID_ARG (shapes, pointers, alignment, overlap of o with
+ * inputs), RKV_ERR_UNSUPPORTED (RoPE position range too large for the on-chip
+ * cos/sin table, D != 128), RKV_ERR_CUDA.  A device-side wait that exceeds
+ * its time limit makes the kernel stop early and record RKV_ERR_TIMEOUT in the
+ * workspace; rkv_attn_status() reads it back.
+ */
+size_t attn_fwd_varlen_workspace_size(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H,
+                                      int32_t D);
+rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                           float softmax_scale, const rkv_rope3d* rope, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * rkv_attn_status -- synchronise `stream` and return the device status word
+ * an earlier attn_fwd_varlen left in `workspace` (RKV_OK or RKV_ERR_TIMEOUT),
+ * then clear it.
+ */
+rkv_status rkv_attn_status(void* workspace, void* stream);
+
+/*
+ * Per-layer rolling KV cache.
+ *
+ * Source: every layer reads and writes a rolling KV cache, and frames are
+ * generated and evicted in a sliding window ("Amazon and Reactor tune Trainium
+ * for real-time video generation", section "Three problems for generic
+ * compilers"; a dedicated per-layer cache-copy kernel: "Optimizing Real-Time
+ * Video Generation on Trainium Chips", item 6 "Neuron Kernel Interface").
+ *
+ * Layout: k and v are device bf16 [slots][tokens_per_frame][H][D], contiguous.
+ * `head` = slot the next frame goes to; `count` = valid frames (0..slots).
+ * Logical frame j (0 = oldest valid) lives in slot (head - count + j) mod slots.
+ */
+typedef struct {
+  void* k;
+  void* v;
+  int32_t slots;
+  int32_t tokens_per_frame;
+  int32_t H;
+  int32_t D;
+  int32_t head;  /* updated by kvcache_ring_update (host side) */
+  int32_t count; /* updated by kvcache_ring_update (host side) */
+} rkv_ring;
+
+/*
+ * kvcache_ring_update -- insert n_frames whole frames of K and V.
+ *
+ *   ring           caller's ring; head/count are updated on success
+ *   k_new, v_new   device bf16 [n_frames * tokens_per_frame][H][D] with row
+ *                  stride new_row_stride (elements); must not overlap the ring
+ *   n_frames       0..slots (0 = no-op)
+ *   n_evicted      optional out: frames dropped = max(0, count + n - slots)
+ * Frame i goes to slot (head + i) mod slots; then head = (head + n) mod slots,
+ * count = min(slots, count + n).  Evicted frames are overwritten, not
+ * cleared: no bytes move for eviction.
+ * Errors: RKV_ERR_INVALID_ARG (n_frames > slots or < 0, null pointers,
+ * head/count out of range, D != 128, misalignment, overlap).
+ */
+rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_new,
+                               int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
+                               void* stream);
+
+/* Slot of logical frame j (0 = oldest valid), or -1 when j is not a valid
+ * frame or the ring is malformed. */
+int32_t rkv_ring_slot(const rkv_ring* ring, int32_t logical_frame);
+
+/* Text of the last error returned on the calling thread ("" if none). */
+const char* rkv_last_error_string(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t rkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKV_H */

@@ -7,18 +7,19 @@ binding name loads the library and raises if it has not been built (there is no
 CPU fallback).
 """
 
-__all__ = ["rkv", "synth"]
+import importlib
+
+_SUBMODULES = ("rkv", "synth", "build")
+__all__ = list(_SUBMODULES)
 
 
 def __getattr__(name):
-    if name == "rkv":
-        from . import rkv
-        return rkv
-    if name == "synth":
-        from . import synth
-        return synth
-    from . import rkv
+    if name.startswith("__"):
+        raise AttributeError(name)
+    if name in _SUBMODULES:
+        return importlib.import_module(f"{__name__}.{name}")
+    rkv = importlib.import_module(f"{__name__}.rkv")
     try:
         return getattr(rkv, name)
     except AttributeError:
-        raise AttributeError(f"module 'rolling_kv_cache_rope_b200' has no attribute {name!r}") from None
+        raise AttributeError(f"module {__name__!r} has no attribute {name!r}") from None

@@ -1,0 +1,745 @@
+// Fused 3D-RoPE + softmax attention for sm_100a (B200), variable-length
+// sequences and frame-block-causal masking, one persistent launch.
+//
+// What it computes (per sequence s, head h):
+//   O = softmax(mask(RoPE(Q) RoPE(K)^T * scale)) V
+// Source: SDPA from a 23,400-token query window to a 32,760-token context,
+// 12 heads, ~70% of compute ("A kernel-centric path to real-time video
+// generation on Trainium", ai4snews summary, second paragraph); attention
+// transposes folded into the attention kernel and a dedicated 3D-RoPE step
+// ("Amazon and Reactor tune Trainium for real-time video generation", sections
+// "Three problems for generic compilers" and "Results with the Neuron Kernel
+// Interface"); the denoise and cache-update passes batched into one run
+// ("Optimizing Real-Time Video Generation on Trainium Chips", item 8 "Model
+// structure optimizations").
+//
+// Design (one CTA per SM, 15 warps):
+//   warps 0-3   softmax for Q sub-tile 0 (one TMEM lane = one query row each)
+//   warps 4-7   softmax for Q sub-tile 1
+//   warps 8-11  RoPE: rotate the Q sub-tiles and each K tile in shared memory
+//               right after TMA lands them, before the tensor core reads them
+//   warp 12     TMA producer for Q and K;  warp 14  TMA producer for V
+//   warp 13     allocates TMEM; one lane issues every tcgen05.mma
+// A work unit is (sequence, head, 256 query rows).  Q/K/V are read straight
+// from token-major [L][H][128] tensors through 3-D TMA descriptors (head is a
+// coordinate), so no transpose pass exists.  S = Q K^T (128x128 fp32) and the
+// running O (128x128 fp32) of both sub-tiles live in TMEM (4 x 128 columns).
+// Softmax reads S with tcgen05.ld, writes P as bf16 back into the first 64
+// columns of the same S region, and the PV MMA takes P straight from TMEM.
+// While one softmax warpgroup works, the tensor core runs the other
+// sub-tile's MMAs (ping-pong).  The running max is only moved (and O rescaled
+// in TMEM) when it grows by more than 2^8, which after the first tile almost
+// never happens.  All waits are bounded; a stuck wait makes every role stop,
+// records RKV_ERR_TIMEOUT in the workspace and frees TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <utility>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace rkv {
+rkv_status check_rope(const rkv_rope3d* rope, int32_t D);
+
+namespace attn {
+
+constexpr int kBM = 128;             // query rows per sub-tile
+constexpr int kSub = 2;              // sub-tiles per unit
+constexpr int kUnitRows = kBM * kSub;
+constexpr int kBN = 128;             // keys per K/V tile
+constexpr int kHD = 128;             // head dim
+constexpr int kStages = 2;           // K and V pipeline depth
+constexpr int kTileBytes = kBN * kHD * 2;      // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2;     // 128 rows x 64 cols
+constexpr int kThreads = 15 * 32;
+constexpr int kMaxTab = 3072;        // cos/sin entries (float2) in shared memory
+constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growth
+
+// shared-memory map (offsets from a 1024-byte aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kSub * kTileBytes;
+constexpr int kOffV = kOffK + kStages * kTileBytes;
+constexpr int kOffTab = kOffV + kStages * kTileBytes;
+constexpr int kOffBar = kOffTab + kMaxTab * 8;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;   // + alignment slack
+
+// TMEM columns: S of sub-tile b at 128*b, O of sub-tile b at 256 + 128*b
+__host__ __device__ constexpr uint32_t col_s(int b) { return 128u * uint32_t(b); }
+__host__ __device__ constexpr uint32_t col_o(int b) { return 256u + 128u * uint32_t(b); }
+constexpr uint32_t kTmemCols = 512;
+
+struct SeqDev {
+  CUtensorMap tq, tk, tv;
+  uint8_t* o;
+  int64_t o_stride_bytes;
+  int32_t Lq, Lk, q_t0, k_t0, q_frame_offset, block_frames;
+  uint32_t flags;
+  int32_t n_qblocks;
+  int32_t unit_begin;
+};
+
+struct Params {
+  SeqDev seq[RKV_MAX_SEQS];
+  int32_t n_seqs, H, total_units;
+  float scale_log2;
+  int32_t grid_h, grid_w, pt, ph, pw;
+  int32_t t_lo, n_t;
+  int32_t tab_base_h, tab_base_w, tab_entries;
+  uint32_t F;
+  FastDiv div_F, div_W;
+  double log2_theta;
+  int32_t* status;
+  uint64_t timeout_ns;
+};
+
+// barrier indices
+enum : int {
+  B_QFULL = 0, B_QREADY, B_QFREE,
+  B_KFULL, B_KREADY = B_KFULL + kStages, B_KFREE = B_KREADY + kStages,
+  B_VFULL = B_KFREE + kStages, B_VFREE = B_VFULL + kStages,
+  B_SFULL = B_VFREE + kStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_OFREE = B_ODONE + 2,
+  B_FINAL = B_OFREE + 2, B_COUNT
+};
+static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
+
+struct Ctx {
+  uint32_t bar0;         // shared address of barrier 0
+  volatile int* abort;   // CTA-wide stop flag
+  const Params* p;
+};
+
+__device__ __forceinline__ uint32_t bar(const Ctx& c, int i) { return c.bar0 + 8u * uint32_t(i); }
+
+// Bounded wait on an mbarrier phase.  Returns false when the CTA is stopping
+// (this or another thread gave up); the first thread to time out records the
+// status word.
+__device__ __noinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t parity, int where) {
+  if (ptx::mbar_try_wait(b, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (ptx::mbar_try_wait(b, parity)) return true;
+    if ((++spins & 31u) == 0) {
+      if (*c.abort) return false;
+      if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
+        *c.abort = 1;
+        atomicCAS(c.p->status, 0, int(RKV_ERR_TIMEOUT) | (where << 8));
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform variant for roles whose 32 lanes continue together.
+__device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t b, uint32_t parity, int where) {
+  const bool ok = wait_phase(c, b, parity, where);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct Unit {
+  int si, head, qb, nkt;
+};
+
+__device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p, int row) {
+  if (s.block_frames <= 0) return s.Lk;
+  const int64_t qf = int64_t(s.q_frame_offset) + row / int64_t(p.F);
+  const int64_t blk = qf / s.block_frames;
+  const int64_t lim = (blk + 1) * s.block_frames * int64_t(p.F);
+  return lim < s.Lk ? lim : s.Lk;
+}
+
+__device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
+  Unit r;
+  int si = 0;
+  while (si + 1 < p.n_seqs && u >= p.seq[si + 1].unit_begin) ++si;
+  const SeqDev& s = p.seq[si];
+  const int local = u - s.unit_begin;
+  const int ord = local / p.H;
+  r.si = si;
+  r.head = local - ord * p.H;
+  r.qb = s.block_frames > 0 ? (s.n_qblocks - 1 - ord) : ord;
+  int last = (r.qb + 1) * kUnitRows - 1;
+  if (last > s.Lq - 1) last = s.Lq - 1;
+  const int64_t kv = row_kv_limit(s, p, last);
+  r.nkt = int((kv + kBN - 1) / kBN);
+  return r;
+}
+
+// ---- RoPE of one 128-row tile in shared memory (128B-swizzled, 2 halves) ----
+// Thread rt (0..127) handles 16-byte chunk (rt & 7) of rows (rt >> 3) + 16k,
+// k = 0..7, in both 64-column halves: 4 rotary pairs per chunk.
+__device__ __forceinline__ void rope_tile(const Params& p, const float2* tab, uint8_t* tile, int row0, int limit,
+                                          int t0, int rt) {
+  const int q = rt & 7;
+#pragma unroll 1
+  for (int k = 0; k < 8; ++k) {
+    const int rr = (rt >> 3) + 16 * k;
+    const int row = row0 + rr;
+    if (row >= limit) continue;
+    const uint32_t f = fdiv(uint32_t(row), p.div_F);
+    const uint32_t in_f = uint32_t(row) - f * p.F;
+    const uint32_t hh = fdiv(in_f, p.div_W);
+    const uint32_t ww = in_f - hh * uint32_t(p.grid_w);
+    const int ti = (t0 + int(f) - p.t_lo) * p.pt;
+    const int hi = p.tab_base_h + int(hh) * p.ph - p.pt;
+    const int wi = p.tab_base_w + int(ww) * p.pw - p.pt - p.ph;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint4* ptr = reinterpret_cast<uint4*>(tile + c * kHalfBytes + rr * 128 + ((q ^ (rr & 7)) << 4));
+      uint4 v = *ptr;
+      uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      const int p0 = c * 32 + q * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int pr = p0 + e;
+        const int idx = pr < p.pt ? ti + pr : (pr < p.pt + p.ph ? hi + pr : wi + pr);
+        const float2 cs = tab[idx];
+        const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+        const float y0 = fmaf(x0, cs.x, -x1 * cs.y);
+        const float y1 = fmaf(x0, cs.y, x1 * cs.x);
+        w4[e] = pack_bf16x2(y0, y1);
+      }
+      *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+}
+
+// Row max of one S tile (raw scores); columns >= lim are hidden when MASKED.
+template <bool MASKED>
+__device__ __forceinline__ float tile_rowmax(uint32_t tS, int lim) {
+  uint32_t r[32];
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    ptx::tmem_ld32(tS + ch * 32, r);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float v = __uint_as_float(r[i]);
+      if (MASKED && ch * 32 + i >= lim) v = -INFINITY;
+      mx[i & 3] = fmaxf(mx[i & 3], v);
+    }
+  }
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// P = exp2(S*scale_log2 - m) as bf16 into the first 64 columns of the S
+// region (P of columns 32c.. goes to packed columns 16c.., which the loop has
+// already read); returns the row sum of the fp32 P values.
+template <bool MASKED>
+__device__ __forceinline__ float tile_exp_store(uint32_t tS, int lim, float scale_log2, float m_use) {
+  uint32_t r[32];
+  float acc[2] = {0.f, 0.f};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    ptx::tmem_ld32(tS + ch * 32, r);
+    ptx::tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float p0 = ptx::ex2_approx(fmaf(__uint_as_float(r[2 * i]), scale_log2, -m_use));
+      float p1 = ptx::ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), scale_log2, -m_use));
+      if (MASKED && ch * 32 + 2 * i >= lim) p0 = 0.f;
+      if (MASKED && ch * 32 + 2 * i + 1 >= lim) p1 = 0.f;
+      acc[i & 1] += p0 + p1;
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    ptx::tmem_st16(tS + ch * 16, pk);
+  }
+  return acc[0] + acc[1];
+}
+
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
+  return ptx::smem_desc_sw128(tile + uint32_t(kk >> 2) * kHalfBytes + uint32_t(kk & 3) * 32u, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk) {
+  return ptx::smem_desc_sw128(tile + uint32_t(kk) * 2048u, kHalfBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8);
+  int* abort_flag = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 4);
+  float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
+  Ctx c;
+  c.bar0 = sbase + kOffBar;
+  c.abort = abort_flag;
+  c.p = &p;
+
+  if (tid == 0) {
+    ptx::mbar_init(bar(c, B_QFULL), 1);
+    ptx::mbar_init(bar(c, B_QREADY), 128);
+    ptx::mbar_init(bar(c, B_QFREE), 1);
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(bar(c, B_KFULL + s), 1);
+      ptx::mbar_init(bar(c, B_KREADY + s), 128);
+      ptx::mbar_init(bar(c, B_KFREE + s), 1);
+      ptx::mbar_init(bar(c, B_VFULL + s), 1);
+      ptx::mbar_init(bar(c, B_VFREE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(c, B_SFULL + b), 1);
+      ptx::mbar_init(bar(c, B_PFULL + b), 128);
+      ptx::mbar_init(bar(c, B_ODONE + b), 1);
+      ptx::mbar_init(bar(c, B_OFREE + b), 128);
+    }
+    ptx::mbar_init(bar(c, B_FINAL), 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 13) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  // cos/sin table (fp64 sincos rounded to fp32) for every reachable position
+  for (int e = tid; e < p.tab_entries; e += kThreads) {
+    int pos, i, n;
+    if (e < p.tab_base_h) {
+      const int ft = e / p.pt;
+      i = e - ft * p.pt; n = p.pt; pos = p.t_lo + ft;
+    } else if (e < p.tab_base_w) {
+      const int hh = (e - p.tab_base_h) / p.ph;
+      i = (e - p.tab_base_h) - hh * p.ph; n = p.ph; pos = hh;
+    } else {
+      const int ww = (e - p.tab_base_w) / p.pw;
+      i = (e - p.tab_base_w) - ww * p.pw; n = p.pw; pos = ww;
+    }
+    double s, co;
+    sincos(double(pos) * exp2(-(double(i) / double(n)) * p.log2_theta), &s, &co);
+    tab[e] = make_float2(__double2float_rn(co), __double2float_rn(s));
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV;
+
+  if (warp < 8) {
+    // ===================== softmax (two warpgroups) =====================
+    const int wg = warp >> 2;
+    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem_base + lane_off + col_s(wg);
+    const uint32_t tO = tmem_base + lane_off + col_o(wg);
+    const float scale_log2 = p.scale_log2;
+    uint32_t g = 0;
+    for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const SeqDev& s = p.seq[un.si];
+      const int qrow = un.qb * kUnitRows + wg * kBM + 32 * (warp & 3) + lane;
+      const int64_t my_limit = row_kv_limit(s, p, qrow < s.Lq ? qrow : s.Lq - 1);
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < un.nkt; ++j, ++g) {
+        if (!wait_warp(c, bar(c, B_SFULL + wg), g & 1u, 1)) goto done;
+        ptx::tc_fence_after();
+        const int64_t kbase = int64_t(j) * kBN;
+        const int lim = kbase + kBN > my_limit ? int(my_limit - kbase) : kBN;
+        const bool masked = __any_sync(0xffffffffu, lim < kBN);
+        const float mx = masked ? tile_rowmax<true>(tS, lim) : tile_rowmax<false>(tS, lim);
+        const float m_new = fmaxf(m, mx * scale_log2);
+        const bool need = m_new > m + kRescaleLog2;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds tiles 0..j-1: wait for the last PV, then rescale in TMEM
+          if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 2)) goto done;
+          ptx::tc_fence_after();
+          const float f = need ? ptx::ex2_approx(m - m_new) : 1.0f;
+          uint32_t r[32];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            ptx::tmem_ld32(tO + ch * 32, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+            ptx::tmem_st32(tO + ch * 32, r);
+          }
+          ptx::tmem_wait_st();
+          l *= f;
+        }
+        if (need) m = m_new;
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        l += masked ? tile_exp_store<true>(tS, lim, scale_log2, m_use)
+                    : tile_exp_store<false>(tS, lim, scale_log2, m_use);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(c, B_PFULL + wg));
+      }
+      // epilogue: O / l -> bf16 -> global (row-major [Lq][H][128])
+      if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 3)) goto done;
+      ptx::tc_fence_after();
+      {
+        const float inv = l > 0.f ? 1.0f / l : 0.f;
+        uint32_t r[32];
+        uint8_t* orow = s.o + int64_t(qrow) * s.o_stride_bytes + int64_t(un.head) * (kHD * 2);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          ptx::tmem_ld32(tO + ch * 32, r);
+          ptx::tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          if (qrow < s.Lq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 64);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(c, B_OFREE + wg));
+    }
+  } else if (warp < 12) {
+    // ===================== RoPE warpgroup =====================
+    const int rt = tid - 256;
+    uint32_t it = 0, ul = 0;
+    for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ul) {
+      const Unit un = decode_unit(p, u);
+      const SeqDev& s = p.seq[un.si];
+      if (!wait_warp(c, bar(c, B_QFULL), ul & 1u, 4)) goto done;
+      if (s.flags & RKV_ROPE_Q) {
+        for (int b = 0; b < kSub; ++b)
+          rope_tile(p, tab, smem + kOffQ + b * kTileBytes, un.qb * kUnitRows + b * kBM, s.Lq, s.q_t0, rt);
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(bar(c, B_QREADY));
+      for (int j = 0; j < un.nkt; ++j, ++it) {
+        const uint32_t st = it % kStages, n = it / kStages;
+        if (!wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5)) goto done;
+        if (s.flags & RKV_ROPE_K) rope_tile(p, tab, smem + kOffK + st * kTileBytes, j * kBN, s.Lk, s.k_t0, rt);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(c, B_KREADY + st));
+      }
+    }
+  } else if (warp == 12) {
+    // ===================== TMA producer: Q and K =====================
+    if (lane == 0) {
+      for (int i = 0; i < p.n_seqs; ++i) {
+        ptx::tma_prefetch_desc(&p.seq[i].tq);
+        ptx::tma_prefetch_desc(&p.seq[i].tk);
+      }
+      uint32_t it = 0, ul = 0;
+      for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ul) {
+        const Unit un = decode_unit(p, u);
+        const SeqDev& s = p.seq[un.si];
+        if (!wait_phase(c, bar(c, B_QFREE), (ul & 1u) ^ 1u, 6)) break;
+        ptx::mbar_expect_tx(bar(c, B_QFULL), kSub * kTileBytes);
+        for (int b = 0; b < kSub; ++b)
+          for (int h2 = 0; h2 < 2; ++h2)
+            ptx::tma_load_3d(sQ + b * kTileBytes + h2 * kHalfBytes, &s.tq, bar(c, B_QFULL), h2 * 64, un.head,
+                             un.qb * kUnitRows + b * kBM);
+        bool ok = true;
+        for (int j = 0; j < un.nkt; ++j, ++it) {
+          const uint32_t st = it % kStages, n = it / kStages;
+          if (!wait_phase(c, bar(c, B_KFREE + st), (n & 1u) ^ 1u, 7)) { ok = false; break; }
+          ptx::mbar_expect_tx(bar(c, B_KFULL + st), kTileBytes);
+          for (int h2 = 0; h2 < 2; ++h2)
+            ptx::tma_load_3d(sK + st * kTileBytes + h2 * kHalfBytes, &s.tk, bar(c, B_KFULL + st), h2 * 64, un.head,
+                             j * kBN);
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 14) {
+    // ===================== TMA producer: V =====================
+    if (lane == 0) {
+      for (int i = 0; i < p.n_seqs; ++i) ptx::tma_prefetch_desc(&p.seq[i].tv);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        const SeqDev& s = p.seq[un.si];
+        for (int j = 0; j < un.nkt; ++j, ++it) {
+          const uint32_t st = it % kStages, n = it / kStages;
+          if (!wait_phase(c, bar(c, B_VFREE + st), (n & 1u) ^ 1u, 8)) { ok = false; break; }
+          ptx::mbar_expect_tx(bar(c, B_VFULL + st), kTileBytes);
+          for (int h2 = 0; h2 < 2; ++h2)
+            ptx::tma_load_3d(sV + st * kTileBytes + h2 * kHalfBytes, &s.tv, bar(c, B_VFULL + st), h2 * 64, un.head,
+                             j * kBN);
+        }
+      }
+    }
+  } else if (warp == 13) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      const uint32_t id_s = ptx::idesc_bf16_f32(kBM, kBN, false);
+      const uint32_t id_pv = ptx::idesc_bf16_f32(kBM, kHD, true);
+      uint32_t it = 0, g = 0, ul = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+        const Unit un = decode_unit(p, u);
+        if (!wait_phase(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
+        ptx::tc_fence_after();
+        for (int j = 0; j < un.nkt; ++j, ++it, ++g) {
+          const uint32_t st = it % kStages, n = it / kStages;
+          if (!wait_phase(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t kt = sK + st * kTileBytes;
+          if (j > 0) {
+            const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
+            if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 11)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t vt = sV + sp * kTileBytes;
+            for (int b = 0; b < kSub && ok; ++b) {
+              if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 12)) { ok = false; break; }
+              ptx::tc_fence_after();
+              if (j == 1) {
+                if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 13)) { ok = false; break; }
+                ptx::tc_fence_after();
+              }
+              // O_b (+)= P_b(j-1) V(j-1): P from TMEM, V from shared memory (MN-major)
+              for (int kk = 0; kk < 8; ++kk)
+                ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, desc_v(vt, kk), id_pv,
+                            (j > 1 || kk > 0) ? 1u : 0u);
+              ptx::mma_commit(bar(c, B_ODONE + b));
+              // S_b(j) = Q_b K(j)^T
+              const uint32_t qt = sQ + b * kTileBytes;
+              for (int kk = 0; kk < 8; ++kk)
+                ptx::mma_ss(tmem_base + col_s(b), desc_kmajor(qt, kk), desc_kmajor(kt, kk), id_s, kk > 0 ? 1u : 0u);
+              ptx::mma_commit(bar(c, B_SFULL + b));
+            }
+            if (!ok) break;
+            ptx::mma_commit(bar(c, B_VFREE + sp));
+          } else {
+            for (int b = 0; b < kSub; ++b) {
+              const uint32_t qt = sQ + b * kTileBytes;
+              for (int kk = 0; kk < 8; ++kk)
+                ptx::mma_ss(tmem_base + col_s(b), desc_kmajor(qt, kk), desc_kmajor(kt, kk), id_s, kk > 0 ? 1u : 0u);
+              ptx::mma_commit(bar(c, B_SFULL + b));
+            }
+          }
+          ptx::mma_commit(bar(c, B_KFREE + st));
+          if (j == un.nkt - 1) ptx::mma_commit(bar(c, B_QFREE));
+        }
+        if (!ok) break;
+        // PV of the unit's last tile
+        const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
+        if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 14)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t vt = sV + sp * kTileBytes;
+        for (int b = 0; b < kSub && ok; ++b) {
+          if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 15)) { ok = false; break; }
+          ptx::tc_fence_after();
+          if (un.nkt == 1) {
+            if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 16)) { ok = false; break; }
+            ptx::tc_fence_after();
+          }
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, desc_v(vt, kk), id_pv,
+                        (un.nkt > 1 || kk > 0) ? 1u : 0u);
+          ptx::mma_commit(bar(c, B_ODONE + b));
+        }
+        if (!ok) break;
+        ptx::mma_commit(bar(c, B_VFREE + sp));
+      }
+      // every tcgen05 op this thread issued is complete before TMEM is freed
+      ptx::mma_commit(bar(c, B_FINAL));
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!ptx::mbar_try_wait(bar(c, B_FINAL), 0)) {
+        if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) break;
+      }
+    }
+  }
+done:
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [L][H][128] bf16 view, row stride in elements; box = 128 rows x 1 head x 64 cols.
+static rkv_status make_map(CUtensorMap* m, const void* ptr, int64_t L, int H, int64_t row_stride) {
+  auto fn = encode_fn();
+  if (!fn) return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(kHD), cuuint64_t(H), cuuint64_t(L)};
+  cuuint64_t strides[2] = {cuuint64_t(kHD * 2), cuuint64_t(row_stride * 2)};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return RKV_OK;
+}
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+constexpr size_t kWorkspaceBytes = 256;
+
+}  // namespace attn
+}  // namespace rkv
+
+using namespace rkv;
+using namespace rkv::attn;
+
+extern "C" size_t attn_fwd_varlen_workspace_size(const rkv_attn_seq*, int32_t, int32_t, int32_t) {
+  return kWorkspaceBytes;
+}
+
+static rkv_status validate_seq(const rkv_attn_seq& s, int i, int32_t H) {
+  const int64_t row = int64_t(H) * kHD;
+  if (!s.q || !s.k || !s.v || !s.o) return fail(RKV_ERR_INVALID_ARG, "seq %d: NULL tensor pointer", i);
+  if (!aligned16(s.q) || !aligned16(s.k) || !aligned16(s.v) || !aligned16(s.o))
+    return fail(RKV_ERR_INVALID_ARG, "seq %d: tensors must be 16-byte aligned", i);
+  if (s.Lq < 1 || s.Lk < 1) return fail(RKV_ERR_INVALID_ARG, "seq %d: Lq and Lk must be >= 1", i);
+  const int64_t st[4] = {s.q_stride, s.k_stride, s.v_stride, s.o_stride};
+  for (int j = 0; j < 4; ++j) {
+    if (st[j] < row) return fail(RKV_ERR_INVALID_ARG, "seq %d: row stride < H*D", i);
+    if ((st[j] * 2) % 16) return fail(RKV_ERR_INVALID_ARG, "seq %d: rows must be 16-byte aligned", i);
+    if (st[j] * 2 >= (int64_t(1) << 40)) return fail(RKV_ERR_INVALID_ARG, "seq %d: row stride too large", i);
+  }
+  if (s.block_frames < 0) return fail(RKV_ERR_INVALID_ARG, "seq %d: block_frames < 0", i);
+  if (s.block_frames > 0 && s.q_frame_offset < 0)
+    return fail(RKV_ERR_INVALID_ARG, "seq %d: q_frame_offset must be >= 0 with a mask", i);
+  if (s.flags & ~(RKV_ROPE_Q | RKV_ROPE_K)) return fail(RKV_ERR_INVALID_ARG, "seq %d: unknown flags", i);
+  if (s.reserved != 0) return fail(RKV_ERR_INVALID_ARG, "seq %d: reserved must be 0", i);
+  return RKV_OK;
+}
+
+static uint64_t span_bytes(int64_t L, int64_t stride, int32_t H) { return uint64_t((L - 1) * stride + int64_t(H) * kHD) * 2; }
+
+extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                      float softmax_scale, const rkv_rope3d* rope, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  clear_error();
+  if (!seqs || n_seqs < 1) return fail(RKV_ERR_INVALID_ARG, "need at least one sequence");
+  if (n_seqs > RKV_MAX_SEQS) return fail(RKV_ERR_UNSUPPORTED, "at most %d sequences per launch", RKV_MAX_SEQS);
+  if (H < 1) return fail(RKV_ERR_INVALID_ARG, "H must be >= 1");
+  if (D != kHD) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", D);
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return fail(RKV_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  rkv_status st = check_rope(rope, D);
+  if (st != RKV_OK) return st;
+  if (!workspace || workspace_bytes < kWorkspaceBytes || !aligned16(workspace))
+    return fail(RKV_ERR_INVALID_ARG, "workspace must be >= %zu bytes and 16-byte aligned", kWorkspaceBytes);
+  for (int i = 0; i < n_seqs; ++i) {
+    st = validate_seq(seqs[i], i, H);
+    if (st != RKV_OK) return st;
+  }
+  for (int i = 0; i < n_seqs; ++i) {
+    const uint64_t ob = span_bytes(seqs[i].Lq, seqs[i].o_stride, H);
+    for (int j = 0; j < n_seqs; ++j) {
+      const rkv_attn_seq& t = seqs[j];
+      if (overlaps(seqs[i].o, ob, t.q, span_bytes(t.Lq, t.q_stride, H)) ||
+          overlaps(seqs[i].o, ob, t.k, span_bytes(t.Lk, t.k_stride, H)) ||
+          overlaps(seqs[i].o, ob, t.v, span_bytes(t.Lk, t.v_stride, H)) ||
+          (i != j && overlaps(seqs[i].o, ob, t.o, span_bytes(t.Lq, t.o_stride, H))))
+        return fail(RKV_ERR_INVALID_ARG, "seq %d: output overlaps an input or another output", i);
+    }
+  }
+
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const int64_t F = int64_t(rope->grid_h) * rope->grid_w;
+  // order: longest context first (cheapest-last helps the static schedule)
+  int order[RKV_MAX_SEQS];
+  for (int i = 0; i < n_seqs; ++i) order[i] = i;
+  for (int i = 1; i < n_seqs; ++i)
+    for (int j = i; j > 0 && seqs[order[j]].Lk > seqs[order[j - 1]].Lk; --j) std::swap(order[j], order[j - 1]);
+
+  int64_t t_lo = INT64_MAX, t_hi = INT64_MIN;
+  int64_t units = 0;
+  for (int oi = 0; oi < n_seqs; ++oi) {
+    const rkv_attn_seq& s = seqs[order[oi]];
+    SeqDev& d = p.seq[oi];
+    if ((st = make_map(&d.tq, s.q, s.Lq, H, s.q_stride)) != RKV_OK) return st;
+    if ((st = make_map(&d.tk, s.k, s.Lk, H, s.k_stride)) != RKV_OK) return st;
+    if ((st = make_map(&d.tv, s.v, s.Lk, H, s.v_stride)) != RKV_OK) return st;
+    d.o = static_cast<uint8_t*>(s.o);
+    d.o_stride_bytes = s.o_stride * 2;
+    d.Lq = s.Lq; d.Lk = s.Lk; d.q_t0 = s.q_t0; d.k_t0 = s.k_t0;
+    d.q_frame_offset = s.q_frame_offset; d.block_frames = s.block_frames; d.flags = s.flags;
+    d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;
+    d.unit_begin = int32_t(units);
+    units += int64_t(d.n_qblocks) * H;
+    if (s.flags & RKV_ROPE_Q) {
+      t_lo = std::min<int64_t>(t_lo, s.q_t0);
+      t_hi = std::max<int64_t>(t_hi, int64_t(s.q_t0) + (s.Lq - 1) / F);
+    }
+    if (s.flags & RKV_ROPE_K) {
+      t_lo = std::min<int64_t>(t_lo, s.k_t0);
+      t_hi = std::max<int64_t>(t_hi, int64_t(s.k_t0) + (s.Lk - 1) / F);
+    }
+  }
+  if (units >= (int64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "too many work units");
+  if (t_lo == INT64_MAX) { t_lo = 0; t_hi = -1; }
+  const int64_t n_t = t_hi - t_lo + 1;
+  const int64_t entries = n_t * rope->pairs_t + int64_t(rope->grid_h) * rope->pairs_h + int64_t(rope->grid_w) * rope->pairs_w;
+  if (entries > kMaxTab)
+    return fail(RKV_ERR_UNSUPPORTED, "RoPE positions need %lld cos/sin entries (max %d)", (long long)entries, kMaxTab);
+  p.n_seqs = n_seqs;
+  p.H = H;
+  p.total_units = int32_t(units);
+  p.scale_log2 = float(double(softmax_scale) * 1.4426950408889634);
+  p.grid_h = rope->grid_h; p.grid_w = rope->grid_w;
+  p.pt = rope->pairs_t; p.ph = rope->pairs_h; p.pw = rope->pairs_w;
+  p.t_lo = int32_t(t_lo); p.n_t = int32_t(n_t);
+  p.tab_base_h = int32_t(n_t * rope->pairs_t);
+  p.tab_base_w = p.tab_base_h + rope->grid_h * rope->pairs_h;
+  p.tab_entries = int32_t(entries);
+  p.F = uint32_t(F);
+  p.div_F = make_fastdiv(uint32_t(F));
+  p.div_W = make_fastdiv(uint32_t(rope->grid_w));
+  p.log2_theta = log2(double(rope->theta));
+  p.status = static_cast<int32_t*>(workspace);
+  p.timeout_ns = 2000000000ull;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kWorkspaceBytes, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
+  const int grid = int(std::min<int64_t>(units, sm_count()));
+  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, cs>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  return RKV_OK;
+}
+
+extern "C" rkv_status rkv_attn_status(void* workspace, void* stream) {
+  clear_error();
+  if (!workspace) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the attention status word");
+  if (word == 0) return RKV_OK;
+  e = cudaMemsetAsync(workspace, 0, sizeof(word), cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the attention status word");
+  return fail(rkv_status(word & 0xff), "attention kernel stopped: bounded wait %d timed out", word >> 8);
+}

@@ -1,0 +1,60 @@
+// Host/device helpers shared by the librkv kernels: status plumbing, fast
+// integer division by run-time constants, bf16 packing.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rkv.h"
+
+namespace rkv {
+
+// ---- host: per-thread last-error text ------------------------------------
+void set_error(const char* fmt, ...);
+void clear_error();
+rkv_status fail(rkv_status code, const char* fmt, ...);
+rkv_status cuda_fail(cudaError_t e, const char* what);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte ranges [a, a+na) and [b, b+nb) overlap.
+inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na && nb && x < y + nb && y < x + na;
+}
+
+// ---- unsigned division by a run-time constant -----------------------------
+// floor(n / d) = (umulhi(n, m) + n) >> s for every n < 2^31, with
+// s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1 (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994).
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  uint32_t s = 0;
+  while ((uint64_t(1) << s) < d) ++s;
+  f.s = s;
+  f.m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.m) + n) >> f.s;
+}
+__device__ __forceinline__ uint32_t fmod_(uint32_t n, uint32_t q, const FastDiv& f) { return n - q * f.d; }
+
+// ---- bf16 packing -----------------------------------------------------------
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+}  // namespace rkv

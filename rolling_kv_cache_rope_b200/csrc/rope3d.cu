@@ -1,0 +1,240 @@
+// Standalone 3D rotary position embedding over (t, h, w).
+//
+// Source: "Amazon and Reactor tune Trainium for real-time video generation",
+// section "Three problems for generic compilers" (video RoPE rotates by height,
+// width and time; generic compilation turns it into many tiny transfers) and
+// "Optimizing Real-Time Video Generation on Trainium Chips", item 6 "Neuron
+// Kernel Interface" (a dedicated 3D-RoPE kernel).  Formula: see rkv.h.
+//
+// Design: the op reads and writes every element once, so it is HBM-bound.
+// Each CTA owns a contiguous block of rows; it first builds, in shared memory,
+// the cos/sin table for the positions its rows can reach (fp64 sincos, split
+// into an fp32 hi + lo pair), then streams 16-byte chunks (4 rotary pairs)
+// with four chunks in flight per thread.  The rotation uses fp32 FMA; when the
+// result is small against the inputs (cancellation, ~1e-4 of outputs) it is
+// recomputed with error-free transforms so every output rounds to within one
+// bf16 ulp of the exactly rounded value.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace rkv {
+
+struct RopeArgs {
+  const uint8_t* x;
+  uint8_t* y;
+  int64_t x_stride_bytes, y_stride_bytes;
+  uint32_t L;
+  uint32_t cpr;            // 16-byte chunks per row = H * 16
+  uint32_t rows_per_cta;
+  uint32_t F;              // tokens per frame
+  int32_t t0;
+  int32_t grid_h, grid_w;
+  int32_t pt, ph, pw;      // rotary pairs per axis
+  double log2_theta;
+  FastDiv div_F, div_W, div_cpr;
+};
+
+constexpr int kRopeThreads = 256;
+constexpr int kRopeUnroll = 4;
+constexpr int kRopeMaxEntries = 4096;  // 64 KB of float4 per CTA
+
+struct TabEntry {
+  float c_hi, s_hi, c_lo, s_lo;
+};
+
+// a*(ch+cl) + b*(sh+sl) with error-free products and sum (fp32).
+__device__ __forceinline__ float dot2_exact(float a, float ch, float cl, float b, float sh, float sl) {
+  const float p1 = a * ch;
+  const float e1 = fmaf(a, ch, -p1);
+  const float p2 = b * sh;
+  const float e2 = fmaf(b, sh, -p2);
+  const float s = p1 + p2;
+  const float bb = s - p1;
+  const float e3 = (p1 - (s - bb)) + (p2 - bb);
+  const float lo = (e1 + e2) + (e3 + fmaf(a, cl, b * sl));
+  return s + lo;
+}
+
+__device__ __forceinline__ void rotate_pair(float x0, float x1, const TabEntry& e, float& y0, float& y1) {
+  y0 = fmaf(x0, e.c_hi, -x1 * e.s_hi);
+  y1 = fmaf(x0, e.s_hi, x1 * e.c_hi);
+  const float lim = fmaxf(fabsf(x0), fabsf(x1)) * 0x1p-12f;
+  if (fabsf(y0) < lim) y0 = dot2_exact(x0, e.c_hi, e.c_lo, -x1, e.s_hi, e.s_lo);
+  if (fabsf(y1) < lim) y1 = dot2_exact(x0, e.s_hi, e.s_lo, x1, e.c_hi, e.c_lo);
+}
+
+__global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) {
+  extern __shared__ float4 tab_raw[];
+  TabEntry* tab = reinterpret_cast<TabEntry*>(tab_raw);
+  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
+  if (r0 >= a.L) return;
+  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
+
+  // positions this CTA can reach
+  const uint32_t f_lo = fdiv(r0, a.div_F), f_hi = fdiv(r1 - 1, a.div_F);
+  const int32_t nt = int32_t(f_hi - f_lo) + 1;
+  int32_t h_lo = 0, nh = a.grid_h;
+  if (f_lo == f_hi) {
+    h_lo = int32_t(fdiv(r0 - f_lo * a.F, a.div_W));
+    nh = int32_t(fdiv(r1 - 1 - f_lo * a.F, a.div_W)) - h_lo + 1;
+  }
+  const int32_t base_h = nt * a.pt;
+  const int32_t base_w = base_h + nh * a.ph;
+  const int32_t n_entries = base_w + a.grid_w * a.pw;
+
+  for (int32_t e = threadIdx.x; e < n_entries; e += kRopeThreads) {
+    int32_t pos, i, n;
+    if (e < base_h) {
+      const int32_t ft = e / a.pt;
+      i = e - ft * a.pt; n = a.pt; pos = a.t0 + int32_t(f_lo) + ft;
+    } else if (e < base_w) {
+      const int32_t hh = (e - base_h) / a.ph;
+      i = (e - base_h) - hh * a.ph; n = a.ph; pos = h_lo + hh;
+    } else {
+      const int32_t ww = (e - base_w) / a.pw;
+      i = (e - base_w) - ww * a.pw; n = a.pw; pos = ww;
+    }
+    const double ang = double(pos) * exp2(-(double(i) / double(n)) * a.log2_theta);
+    double s, c;
+    sincos(ang, &s, &c);
+    TabEntry t;
+    t.c_hi = __double2float_rn(c);
+    t.s_hi = __double2float_rn(s);
+    t.c_lo = __double2float_rn(c - double(t.c_hi));
+    t.s_lo = __double2float_rn(s - double(t.s_hi));
+    tab[e] = t;
+  }
+  __syncthreads();
+
+  const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
+  for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
+    uint4 v[kRopeUnroll];
+    uint32_t row[kRopeUnroll], within[kRopeUnroll];
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const uint32_t ci = base + u * kRopeThreads;
+      if (ci < c_end) {
+        row[u] = fdiv(ci, a.div_cpr);
+        within[u] = ci - row[u] * a.cpr;
+        v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(row[u]) * a.x_stride_bytes + uint64_t(within[u]) * 16u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const uint32_t ci = base + u * kRopeThreads;
+      if (ci >= c_end) continue;
+      const uint32_t r = row[u];
+      const uint32_t f = fdiv(r, a.div_F);
+      const uint32_t in_f = r - f * a.F;
+      const uint32_t hh = fdiv(in_f, a.div_W);
+      const uint32_t ww = in_f - hh * uint32_t(a.grid_w);
+      const int32_t ti = int32_t(f - f_lo) * a.pt;
+      const int32_t hi = base_h + (int32_t(hh) - h_lo) * a.ph - a.pt;
+      const int32_t wi = base_w + int32_t(ww) * a.pw - a.pt - a.ph;
+      const int32_t p0 = int32_t(within[u] & 15u) * 4;   // first rotary pair of this chunk
+      uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int32_t p = p0 + k;
+        const int32_t idx = p < a.pt ? ti + p : (p < a.pt + a.ph ? hi + p : wi + p);
+        const TabEntry e = tab[idx];
+        float y0, y1;
+        rotate_pair(bf16lo_to_f32(w4[k]), bf16hi_to_f32(w4[k]), e, y0, y1);
+        w4[k] = pack_bf16x2(y0, y1);
+      }
+      *reinterpret_cast<uint4*>(a.y + int64_t(r) * a.y_stride_bytes + uint64_t(within[u]) * 16u) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+}
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+rkv_status check_rope(const rkv_rope3d* rope, int32_t D) {
+  if (!rope) return fail(RKV_ERR_INVALID_ARG, "rope parameters are NULL");
+  if (rope->grid_h < 1 || rope->grid_w < 1) return fail(RKV_ERR_INVALID_ARG, "grid_h/grid_w must be >= 1");
+  if (int64_t(rope->grid_h) * rope->grid_w >= (int64_t(1) << 30))
+    return fail(RKV_ERR_INVALID_ARG, "frame grid too large");
+  if (rope->pairs_t < 1 || rope->pairs_h < 1 || rope->pairs_w < 1)
+    return fail(RKV_ERR_INVALID_ARG, "pairs per axis must be >= 1");
+  if (rope->pairs_t + rope->pairs_h + rope->pairs_w != D / 2)
+    return fail(RKV_ERR_INVALID_ARG, "pairs_t+pairs_h+pairs_w must equal D/2");
+  if (!(rope->theta > 1.0f) || !isfinite(rope->theta)) return fail(RKV_ERR_INVALID_ARG, "theta must be finite and > 1");
+  return RKV_OK;
+}
+
+}  // namespace rkv
+
+using namespace rkv;
+
+extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H, int32_t D, int64_t x_row_stride,
+                                   int64_t y_row_stride, int32_t t0, const rkv_rope3d* rope, void* stream) {
+  clear_error();
+  if (D != 128) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", D);
+  rkv_status st = check_rope(rope, D);
+  if (st != RKV_OK) return st;
+  if (L < 0 || H < 1) return fail(RKV_ERR_INVALID_ARG, "L must be >= 0 and H >= 1");
+  if (L == 0) return RKV_OK;
+  if (!x || !y) return fail(RKV_ERR_INVALID_ARG, "x/y is NULL");
+  const int64_t row_elems = int64_t(H) * D;
+  if (x_row_stride < row_elems || y_row_stride < row_elems) return fail(RKV_ERR_INVALID_ARG, "row stride < H*D");
+  if (!aligned16(x) || !aligned16(y) || (x_row_stride * 2) % 16 || (y_row_stride * 2) % 16)
+    return fail(RKV_ERR_INVALID_ARG, "rows must be 16-byte aligned");
+  const uint64_t xb = uint64_t((L - 1) * x_row_stride + row_elems) * 2;
+  const uint64_t yb = uint64_t((L - 1) * y_row_stride + row_elems) * 2;
+  if (x != y && overlaps(x, xb, y, yb)) return fail(RKV_ERR_INVALID_ARG, "x and y overlap without being identical");
+  if (x == y && x_row_stride != y_row_stride) return fail(RKV_ERR_INVALID_ARG, "in-place call needs equal strides");
+  if (L >= (int64_t(1) << 31) || uint64_t(L) * H * 16 >= (uint64_t(1) << 31))
+    return fail(RKV_ERR_UNSUPPORTED, "too many rows for one launch");
+  const int64_t last_t = int64_t(t0) + (L - 1) / (int64_t(rope->grid_h) * rope->grid_w);
+  if (last_t > INT32_MAX) return fail(RKV_ERR_INVALID_ARG, "time index overflows int32");
+
+  RopeArgs a;
+  a.x = static_cast<const uint8_t*>(x);
+  a.y = static_cast<uint8_t*>(y);
+  a.x_stride_bytes = x_row_stride * 2;
+  a.y_stride_bytes = y_row_stride * 2;
+  a.L = uint32_t(L);
+  a.cpr = uint32_t(H) * 16u;
+  a.F = uint32_t(rope->grid_h) * uint32_t(rope->grid_w);
+  a.t0 = t0;
+  a.grid_h = rope->grid_h;
+  a.grid_w = rope->grid_w;
+  a.pt = rope->pairs_t;
+  a.ph = rope->pairs_h;
+  a.pw = rope->pairs_w;
+  a.log2_theta = log2(double(rope->theta));
+  a.div_F = make_fastdiv(a.F);
+  a.div_W = make_fastdiv(uint32_t(rope->grid_w));
+  a.div_cpr = make_fastdiv(a.cpr);
+  const int64_t target_ctas = int64_t(sm_count()) * 4;
+  int64_t rpc = (L + target_ctas - 1) / target_ctas;
+  if (rpc < 1) rpc = 1;
+  // keep the per-CTA table within budget: shrink the row block if needed
+  auto entries = [&](int64_t rows) {
+    const int64_t nt = rows / a.F + 2;
+    return nt * a.pt + int64_t(a.grid_h) * a.ph + int64_t(a.grid_w) * a.pw;
+  };
+  if (int64_t(a.grid_w) * a.pw + 2 * a.pt + int64_t(a.grid_h) * a.ph > kRopeMaxEntries)
+    return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
+  while (rpc > 1 && entries(rpc) > kRopeMaxEntries) rpc = (rpc + 1) / 2;
+  a.rows_per_cta = uint32_t(rpc);
+  const int64_t grid = (L + rpc - 1) / rpc;
+  const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kRopeMaxEntries * int(sizeof(TabEntry)));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
+    attr_set = true;
+  }
+  rope3d_kernel<<<uint32_t(grid), kRopeThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
+  return RKV_OK;
+}

@@ -1,0 +1,181 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects invalid arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_]\w*\s*\*?\s+\*?([A-Za-z_]\w*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "return")))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("rope3d_apply", "attn_fwd_varlen", "kvcache_ring_update"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    lib = ctypes.CDLL(lib_path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+@pytest.fixture(scope="module")
+def rkv(lib_path):
+    from rolling_kv_cache_rope_b200 import rkv as m
+    return m
+
+
+def fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_version(rkv):
+    assert rkv.rkv_version() >= 100
+
+
+def ring(rkv, slots=5, F=24, H=2, D=128, head=0, count=0, k=0x10000, v=0x20000000):
+    return rkv.rkv_ring(k, v, slots, F, H, D, head, count)
+
+
+def test_ring_slot_host_logic(rkv):
+    lib = rkv.lib()
+    r = ring(rkv, slots=5, head=1, count=5)
+    assert [lib.rkv_ring_slot(ctypes.byref(r), j) for j in range(6)] == [1, 2, 3, 4, 0, -1]
+    r = ring(rkv, slots=5, head=3, count=3)
+    assert [lib.rkv_ring_slot(ctypes.byref(r), j) for j in range(4)] == [0, 1, 2, -1]
+    assert lib.rkv_ring_slot(ctypes.byref(r), -1) == -1
+    bad = ring(rkv, slots=5, head=7, count=3)
+    assert lib.rkv_ring_slot(ctypes.byref(bad), 0) == -1
+    assert lib.rkv_ring_slot(None, 0) == -1
+
+
+@pytest.mark.parametrize("change,n,frag", [
+    (dict(), 6, "n_frames"),                 # more frames than slots
+    (dict(), -1, "n_frames"),
+    (dict(D=64), 1, "128"),
+    (dict(head=5), 1, "head"),
+    (dict(count=9), 1, "count"),
+    (dict(k=0), 1, "NULL"),
+    (dict(k=0x10008), 1, "aligned"),
+    (dict(v=0x10000), 1, "overlap"),         # k and v buffers overlap
+])
+def test_ring_update_rejects(rkv, change, n, frag):
+    lib = rkv.lib()
+    r = ring(rkv, **change)
+    before = (r.head, r.count)
+    ev = ctypes.c_int32(-7)
+    st = lib.kvcache_ring_update(ctypes.byref(r), fake(0x40000000), fake(0x50000000), 2 * 128, n,
+                                 ctypes.byref(ev), None)
+    assert st == rkv.RKV_ERR_INVALID_ARG
+    assert frag in rkv.rkv_last_error_string()
+    assert (r.head, r.count) == before and ev.value == -7
+
+
+def test_ring_update_rejects_bad_sources(rkv):
+    lib = rkv.lib()
+    r = ring(rkv)
+    for kn, vn, stride in [(0, 0x50000000, 256), (0x40000004, 0x50000000, 256), (0x40000000, 0x50000000, 100),
+                           (0x10000, 0x50000000, 256)]:       # last: k_new overlaps the ring
+        st = lib.kvcache_ring_update(ctypes.byref(r), fake(kn), fake(vn), stride, 2, None, None)
+        assert st == rkv.RKV_ERR_INVALID_ARG, (kn, vn, stride)
+
+
+def test_ring_update_zero_frames_is_a_host_noop(rkv):
+    lib = rkv.lib()
+    r = ring(rkv, head=2, count=4)
+    ev = ctypes.c_int32(-1)
+    assert lib.kvcache_ring_update(ctypes.byref(r), None, None, 256, 0, ctypes.byref(ev), None) == rkv.RKV_OK
+    assert (r.head, r.count, ev.value) == (2, 4, 0)
+
+
+def rope(rkv, **kw):
+    base = dict(grid_h=4, grid_w=6, pairs=(22, 21, 21), theta=10000.0)
+    base.update(kw)
+    return rkv.make_rope(base["grid_h"], base["grid_w"], base["pairs"], base["theta"])
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(D=64), "128"),
+    (dict(x=0), "NULL"),
+    (dict(x=0x1008), "aligned"),
+    (dict(xs=100), "stride"),
+    (dict(y=0x1100), "overlap"),
+    (dict(rope_kw=dict(pairs=(20, 21, 21))), "pairs"),
+    (dict(rope_kw=dict(grid_h=0)), "grid"),
+    (dict(rope_kw=dict(theta=1.0)), "theta"),
+])
+def test_rope_rejects(rkv, args, frag):
+    lib = rkv.lib()
+    a = dict(x=0x1000, y=0x90000000, L=72, H=2, D=128, xs=256, ys=256)
+    a.update({k: v for k, v in args.items() if k != "rope_kw"})
+    r = rope(rkv, **args.get("rope_kw", {}))
+    st = lib.rope3d_apply(fake(a["x"]), fake(a["y"]), a["L"], a["H"], a["D"], a["xs"], a["ys"], 0,
+                          ctypes.byref(r), None)
+    assert st == rkv.RKV_ERR_INVALID_ARG, rkv.rkv_last_error_string()
+    assert frag in rkv.rkv_last_error_string()
+
+
+def test_rope_zero_rows_is_a_noop(rkv):
+    r = rope(rkv)
+    assert rkv.lib().rope3d_apply(None, None, 0, 2, 128, 256, 256, 0, ctypes.byref(r), None) == rkv.RKV_OK
+
+
+def seq(rkv, **kw):
+    base = dict(q=0x100000, k=0x200000, v=0x300000, o=0x400000, q_stride=256, k_stride=256, v_stride=256,
+                o_stride=256, Lq=72, Lk=120, q_t0=2, k_t0=0, q_frame_offset=2, block_frames=0, flags=3,
+                reserved=0)
+    base.update(kw)
+    return rkv.rkv_attn_seq(**base)
+
+
+@pytest.mark.parametrize("kw,frag", [
+    (dict(Lq=0), "Lq"),
+    (dict(k=0), "NULL"),
+    (dict(v=0x300008), "aligned"),
+    (dict(o_stride=128), "stride"),
+    (dict(block_frames=-1), "block_frames"),
+    (dict(block_frames=3, q_frame_offset=-1), "q_frame_offset"),
+    (dict(flags=8), "flags"),
+    (dict(reserved=1), "reserved"),
+    (dict(o=0x100100), "overlaps"),
+])
+def test_attn_rejects(rkv, kw, frag):
+    lib = rkv.lib()
+    arr = (rkv.rkv_attn_seq * 1)(seq(rkv, **kw))
+    r = rope(rkv)
+    st = lib.attn_fwd_varlen(arr, 1, 2, 128, 0.088, ctypes.byref(r), fake(0x700000), 256, None)
+    assert st == rkv.RKV_ERR_INVALID_ARG, rkv.rkv_last_error_string()
+    assert frag in rkv.rkv_last_error_string()
+
+
+def test_attn_rejects_launch_level_arguments(rkv):
+    lib = rkv.lib()
+    arr = (rkv.rkv_attn_seq * 1)(seq(rkv))
+    r = rope(rkv)
+    ws = fake(0x700000)
+    assert lib.attn_fwd_varlen(arr, 0, 2, 128, 0.088, ctypes.byref(r), ws, 256, None) == rkv.RKV_ERR_INVALID_ARG
+    assert lib.attn_fwd_varlen(arr, 1, 2, 64, 0.088, ctypes.byref(r), ws, 256, None) == rkv.RKV_ERR_INVALID_ARG
+    assert lib.attn_fwd_varlen(arr, 1, 2, 128, -1.0, ctypes.byref(r), ws, 256, None) == rkv.RKV_ERR_INVALID_ARG
+    assert lib.attn_fwd_varlen(arr, 1, 2, 128, 0.088, ctypes.byref(r), None, 256, None) == rkv.RKV_ERR_INVALID_ARG
+    assert lib.attn_fwd_varlen(arr, 1, 2, 128, 0.088, ctypes.byref(r), ws, 8, None) == rkv.RKV_ERR_INVALID_ARG
+    many = (rkv.rkv_attn_seq * 17)(*[seq(rkv) for _ in range(17)])
+    assert lib.attn_fwd_varlen(many, 17, 2, 128, 0.088, ctypes.byref(r), ws, 256, None) == rkv.RKV_ERR_UNSUPPORTED
+    assert lib.attn_fwd_varlen_workspace_size(arr, 1, 2, 128) >= 4
+
+
+def test_python_binding_refuses_non_bf16(rkv):
+    import torch
+    x = torch.zeros(4, 2, 128, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        rkv.rope3d_apply(x, rope=rkv.make_rope(4, 6))

@@ -1,0 +1,74 @@
+"""Standalone 3D-RoPE on the GPU vs the fp64 oracle: every output within one
+bf16 ulp of the oracle's correctly rounded value (nearly all identical)."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bf16_bits_to_f64, bf16_ulp_distance, f64_to_bf16_bits, rope3d_ref
+from rolling_kv_cache_rope_b200.synth import DENOISE, MID, TINY, bf16_normal_bits
+from tests._gpu import need_gpu, to_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def check_rope(L, H, grid_h, grid_w, t0, seed, in_place=False, stride_mult=1, pairs=(22, 21, 21)):
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    D = 128
+    xb = bf16_normal_bits(seed, (L, H, D))
+    ref = f64_to_bf16_bits(rope3d_ref(bf16_bits_to_f64(xb), t0, grid_h, grid_w, pairs))
+    rope = rkv.make_rope(grid_h, grid_w, pairs)
+    if stride_mult == 1:
+        x = to_dev(xb)
+    else:
+        wide = np.zeros((L, stride_mult * H, D), dtype=np.uint16)
+        wide[:, :H] = xb
+        x = to_dev(wide)[:, :H, :]
+    y = x if in_place else torch.empty((L, H, D), dtype=torch.bfloat16, device="cuda")
+    rkv.rope3d_apply(x, y, t0=t0, rope=rope)
+    torch.cuda.synchronize()
+    got = to_bits(y)
+    ulp = bf16_ulp_distance(got, ref)
+    assert int(ulp.max()) <= 1, f"max ulp {int(ulp.max())}"
+    exact = float((ulp == 0).mean())
+    assert exact > 0.999, f"only {exact:.5f} of outputs identical to the oracle's rounding"
+    return exact
+
+
+def test_tiny_q_and_k():
+    check_rope(TINY.Lq, TINY.heads, TINY.grid_h, TINY.grid_w, TINY.q_t0, TINY.seed)
+    check_rope(TINY.Lk, TINY.heads, TINY.grid_h, TINY.grid_w, TINY.k_t0, TINY.seed + 1)
+
+
+def test_mid_q_and_k():
+    check_rope(MID.Lq, MID.heads, MID.grid_h, MID.grid_w, MID.q_t0, MID.seed)
+    check_rope(MID.Lk, MID.heads, MID.grid_h, MID.grid_w, MID.k_t0, MID.seed + 1)
+
+
+def test_denoise_q_full_size():
+    check_rope(DENOISE.Lq, DENOISE.heads, DENOISE.grid_h, DENOISE.grid_w, DENOISE.q_t0, DENOISE.seed)
+
+
+def test_denoise_k_full_size():
+    check_rope(DENOISE.Lk, DENOISE.heads, DENOISE.grid_h, DENOISE.grid_w, DENOISE.k_t0, DENOISE.seed + 1)
+
+
+def test_in_place_and_strided():
+    check_rope(1000, 3, 4, 6, 5, 11, in_place=True)
+    check_rope(1000, 3, 4, 6, 5, 12, stride_mult=3)
+    check_rope(777, 2, 15, 26, 0, 13, in_place=True, stride_mult=2)
+
+
+def test_ragged_and_single_row():
+    check_rope(1, 1, 30, 52, 9, 14)
+    check_rope(1561, 12, 30, 52, 3, 15)          # one frame plus one token
+    check_rope(24 * 40 + 7, 2, 4, 6, 35, 16)     # many frames, long time axis
+
+
+def test_other_axis_split():
+    check_rope(300, 2, 5, 7, 1, 17, pairs=(32, 16, 16))
+
+
+def test_large_time_index():
+    check_rope(200, 2, 4, 6, 1000, 18)
