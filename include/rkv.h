@@ -175,6 +175,35 @@ rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, 
 rkv_status rkv_attn_status(void* workspace, void* stream);
 
 /*
+ * attn_fwd_varlen_noalloc -- attn_fwd_varlen without a caller workspace.
+ *
+ * The pages have no counterpart to this call; it exists for callers of this
+ * library that cannot allocate device memory themselves: plugin and custom-op
+ * hosts that hand a kernel only its input and output buffers, engines whose
+ * device memory is fully pre-planned, and code that must not call cudaMalloc
+ * (which can synchronise the device).  The caller still passes every input
+ * and output; the few bytes of scratch the attention launch needs (its status
+ * word, cleared at the start of every call) come from a fixed 256-byte array
+ * inside librkv.so.  Every GPU that loads the library holds that array until
+ * the process exits.  Nothing is allocated by this call.
+ *
+ *   seqs ... stream   as for attn_fwd_varlen
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture on that device.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents.  Calls that overlap on the GPU (on different streams, or
+ * from different host threads without ordering) race on it; serialise them.
+ * Limit: a launch whose scratch need (attn_fwd_varlen_workspace_size) exceeds
+ * 256 bytes is rejected with RKV_ERR_UNSUPPORTED.
+ * A device-side timeout stops the kernel as in attn_fwd_varlen but is only
+ * recorded in the internal array; callers that need it reported back use
+ * attn_fwd_varlen with their own workspace and rkv_attn_status.
+ */
+rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                   float softmax_scale, const rkv_rope3d* rope, void* stream);
+
+/*
  * Per-layer rolling KV cache.
  *
  * Source: every layer reads and writes a rolling KV cache, and frames are

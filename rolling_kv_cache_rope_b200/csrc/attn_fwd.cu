@@ -38,6 +38,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <utility>
 
 #include "common.cuh"
@@ -742,4 +743,58 @@ extern "C" rkv_status rkv_attn_status(void* workspace, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the attention status word");
   return fail(rkv_status(word & 0xff), "attention kernel stopped: bounded wait %d timed out", word >> 8);
+}
+
+// ---------------------------------------------------------------------------
+// attn_fwd_varlen_noalloc: the same launch, with the workspace taken from a
+// fixed device array inside this library instead of caller memory.  For
+// callers that cannot allocate device memory themselves.
+// ---------------------------------------------------------------------------
+namespace rkv {
+namespace attn {
+
+constexpr size_t kNoAllocScratchBytes = 256;  // the whole fixed scratch
+static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "workspace outgrew the fixed scratch");
+constexpr int kMaxDevices = 64;
+
+// Every GPU that loads librkv.so holds this array until the process exits.
+// Host code must not pass its name to a kernel: on the host it is only a
+// stand-in; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and cached.
+static rkv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RKV_ERR_UNSUPPORTED, "device index %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc attention scratch)");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RKV_OK;
+}
+
+}  // namespace attn
+}  // namespace rkv
+
+extern "C" rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                              float softmax_scale, const rkv_rope3d* rope, void* stream) {
+  clear_error();
+  const size_t need = attn_fwd_varlen_workspace_size(seqs, n_seqs, H, D);
+  if (need > kNoAllocScratchBytes)
+    return fail(RKV_ERR_UNSUPPORTED, "this launch needs %zu bytes of scratch; the no-alloc entry point has %zu",
+                need, kNoAllocScratchBytes);
+  void* ws = nullptr;
+  rkv_status st = noalloc_scratch(&ws);
+  if (st != RKV_OK) return st;
+  return attn_fwd_varlen(seqs, n_seqs, H, D, softmax_scale, rope, ws, kNoAllocScratchBytes, stream);
 }
