@@ -49,7 +49,7 @@ rkv_status check_rope(const rkv_rope3d* rope, int32_t D);
 
 namespace attn {
 
-constexpr int kBM = 128;             // query rows per sub-tile
+constexpr int kBM = 128;             // query rows per sub-tile (one TMEM lane each)
 constexpr int kSub = 2;              // sub-tiles per unit
 constexpr int kUnitRows = kBM * kSub;
 constexpr int kBN = 128;             // keys per K/V tile
@@ -57,16 +57,21 @@ constexpr int kHD = 128;             // head dim
 constexpr int kStages = 2;           // K and V pipeline depth
 constexpr int kTileBytes = kBN * kHD * 2;      // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;     // 128 rows x 64 cols
-constexpr int kThreads = 15 * 32;
-constexpr int kMaxTab = 3072;        // cos/sin entries (float2) in shared memory
+constexpr int kThreads = 16 * 32;
+constexpr int kTabEntryBytes = 32;   // cos and sin of 4 consecutive rotary pairs
+constexpr int kMaxTabEntries = 768;  // 24 KB of shared memory (cos array, then sin array)
 constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growth
+// register split (setmaxnreg): two softmax warpgroups, RoPE, producers; the
+// four shares add up to the 4 x 128 registers per thread the block launches with
+constexpr int kRegSoftmax = 168, kRegRope = 96, kRegProducer = 80;
+static_assert(2 * kRegSoftmax + kRegRope + kRegProducer == 4 * 128, "register split must match the launch");
 
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kSub * kTileBytes;
 constexpr int kOffV = kOffK + kStages * kTileBytes;
 constexpr int kOffTab = kOffV + kStages * kTileBytes;
-constexpr int kOffBar = kOffTab + kMaxTab * 8;
+constexpr int kOffBar = kOffTab + kMaxTabEntries * kTabEntryBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;   // + alignment slack
 
 // TMEM columns: S of sub-tile b at 128*b, O of sub-tile b at 256 + 128*b
@@ -88,9 +93,19 @@ struct Params {
   SeqDev seq[RKV_MAX_SEQS];
   int32_t n_seqs, H, total_units;
   float scale_log2;
-  int32_t grid_h, grid_w, pt, ph, pw;
+  int32_t grid_h, grid_w;
   int32_t t_lo, n_t;
-  int32_t tab_base_h, tab_base_w, tab_entries;
+  // RoPE table: entry e holds cos (and, tab_entries entries later, sin) of 4
+  // consecutive global rotary pairs.  Axis a owns entries ax_tab[a] .. as
+  // [chunk k of the axis][position]; chunk k covers global pairs
+  // 4*(ax_chunk0[a] + k) .. +3 (pairs outside the axis hold cos 1, sin 0).
+  int32_t ax_first[3], ax_count[3], ax_chunk0[3], ax_nch[3], ax_npos[3], ax_tab[3];
+  int32_t tab_entries;
+  // per 16-byte chunk g of a head (pairs 4g..4g+3): entry of position 0 on the
+  // axis of its first pair (lo) and of its last pair (hi); axes; and which
+  // of the 4 pairs take the hi axis (0 when the chunk lies on one axis)
+  int32_t ch_base_lo[16], ch_base_hi[16];
+  int8_t ch_ax_lo[16], ch_ax_hi[16], ch_sel[16];
   uint32_t F;
   FastDiv div_F, div_W;
   double log2_theta;
@@ -119,13 +134,13 @@ __device__ __forceinline__ uint32_t bar(const Ctx& c, int i) { return c.bar0 + 8
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is stopping
 // (this or another thread gave up); the first thread to time out records the
 // status word.
-__device__ __noinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t parity, int where) {
+__device__ __forceinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t parity, int where) {
   if (ptx::mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
     if (ptx::mbar_try_wait(b, parity)) return true;
-    if ((++spins & 31u) == 0) {
+    if ((++spins & 15u) == 0) {
       if (*c.abort) return false;
       if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
         *c.abort = 1;
@@ -154,15 +169,19 @@ __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p
   return lim < s.Lk ? lim : s.Lk;
 }
 
+// Units are numbered head-major within a sequence (all query blocks of head 0,
+// then head 1, ...), so the CTAs in flight at any time share the K/V tiles of
+// one or two heads in L2.  Masked sequences list their query blocks from the
+// most to the least visible keys.
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   Unit r;
   int si = 0;
   while (si + 1 < p.n_seqs && u >= p.seq[si + 1].unit_begin) ++si;
   const SeqDev& s = p.seq[si];
   const int local = u - s.unit_begin;
-  const int ord = local / p.H;
   r.si = si;
-  r.head = local - ord * p.H;
+  r.head = local / s.n_qblocks;
+  const int ord = local - r.head * s.n_qblocks;
   r.qb = s.block_frames > 0 ? (s.n_qblocks - 1 - ord) : ord;
   int last = (r.qb + 1) * kUnitRows - 1;
   if (last > s.Lq - 1) last = s.Lq - 1;
@@ -171,88 +190,97 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   return r;
 }
 
-// ---- RoPE of one 128-row tile in shared memory (128B-swizzled, 2 halves) ----
-// Thread rt (0..127) handles 16-byte chunk (rt & 7) of rows (rt >> 3) + 16k,
-// k = 0..7, in both 64-column halves: 4 rotary pairs per chunk.
-__device__ __forceinline__ void rope_tile(const Params& p, const float2* tab, uint8_t* tile, int row0, int limit,
-                                          int t0, int rt) {
-  const int q = rt & 7;
-#pragma unroll 1
-  for (int k = 0; k < 8; ++k) {
-    const int rr = (rt >> 3) + 16 * k;
-    const int row = row0 + rr;
-    if (row >= limit) continue;
-    const uint32_t f = fdiv(uint32_t(row), p.div_F);
-    const uint32_t in_f = uint32_t(row) - f * p.F;
-    const uint32_t hh = fdiv(in_f, p.div_W);
-    const uint32_t ww = in_f - hh * uint32_t(p.grid_w);
-    const int ti = (t0 + int(f) - p.t_lo) * p.pt;
-    const int hi = p.tab_base_h + int(hh) * p.ph - p.pt;
-    const int wi = p.tab_base_w + int(ww) * p.pw - p.pt - p.ph;
+__device__ __forceinline__ int axis_of(const Params& p, int pair) {
+  return pair < p.ax_first[1] ? 0 : (pair < p.ax_first[2] ? 1 : 2);
+}
+
+__device__ __forceinline__ int pick3(int a, int x, int y, int z) { return a == 0 ? x : (a == 1 ? y : z); }
+
+// Rotate 4 rotary pairs (one 16-byte chunk, bf16) by the given cos / sin.
+__device__ __forceinline__ uint4 rotate_chunk(uint4 v, float4 C, float4 S) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint4* ptr = reinterpret_cast<uint4*>(tile + c * kHalfBytes + rr * 128 + ((q ^ (rr & 7)) << 4));
-      uint4 v = *ptr;
-      uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-      const int p0 = c * 32 + q * 4;
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t a = w[2 * h], b = w[2 * h + 1];
+    const float2 x0 = make_float2(bf16lo_to_f32(a), bf16lo_to_f32(b));
+    const float2 x1 = make_float2(bf16hi_to_f32(a), bf16hi_to_f32(b));
+    const float2 nx1 = make_float2(__uint_as_float((a & 0xFFFF0000u) ^ 0x80000000u),
+                                   __uint_as_float((b & 0xFFFF0000u) ^ 0x80000000u));
+    const float2 c = h ? make_float2(C.z, C.w) : make_float2(C.x, C.y);
+    const float2 s = h ? make_float2(S.z, S.w) : make_float2(S.x, S.y);
+    const float2 y0 = __ffma2_rn(x0, c, __fmul2_rn(nx1, s));   // x0 cos - x1 sin
+    const float2 y1 = __ffma2_rn(x0, s, __fmul2_rn(x1, c));    // x0 sin + x1 cos
+    o[2 * h] = pack_bf16x2(y0.x, y1.x);
+    o[2 * h + 1] = pack_bf16x2(y0.y, y1.y);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// RoPE of one 128-row tile in shared memory (128B-swizzled, 2 halves), in
+// place.  Thread rt owns row rt: its (t, h, w) is computed once and it walks
+// the row's 16 chunks (4 rotary pairs each).  Chunk g lies on the same axis
+// for every thread, so all branches are warp-uniform, and neighbouring rows
+// read broadcast (t, h) or adjacent (w) table entries.  Loads for 4 chunks
+// are issued before their arithmetic.
+//
+// A chunk that straddles two axes reads both axes' entries; each axis' table
+// holds cos 1 / sin 0 for pairs outside the axis, so the chunk's cos and sin
+// are the elementwise product of the two cos and the sum of the two sin.
+//
+// kPT/kPH > 0: the axis split is known at compile time (chunk -> axis folds to
+// constants and only straddling chunks load twice); kPT == 0: read it from
+// the parameters.
+template <int kPT, int kPH>
+__device__ __forceinline__ void rope_tile(const Params& p, uint32_t tabC, uint32_t tabS, uint32_t tile, int row0,
+                                          int limit, int t0, int rt) {
+  const int row = row0 + rt;
+  if (row >= limit) return;
+  const uint32_t f = fdiv(uint32_t(row), p.div_F);
+  const uint32_t in_f = uint32_t(row) - f * p.F;
+  const uint32_t hh = fdiv(in_f, p.div_W);
+  const int pt = t0 + int(f) - p.t_lo, ph = int(hh), pw = int(in_f - hh * uint32_t(p.grid_w));
+  const uint32_t row_addr = tile + uint32_t(rt) * 128u;
+  const uint32_t swz = uint32_t(rt & 7);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int pr = p0 + e;
-        const int idx = pr < p.pt ? ti + pr : (pr < p.pt + p.ph ? hi + pr : wi + pr);
-        const float2 cs = tab[idx];
-        const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-        const float y0 = fmaf(x0, cs.x, -x1 * cs.y);
-        const float y1 = fmaf(x0, cs.y, x1 * cs.x);
-        w4[e] = pack_bf16x2(y0, y1);
+  for (int g0 = 0; g0 < 16; g0 += 4) {
+    uint4 v[4];
+    float4 C[4], S[4];
+    uint32_t addr[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int g = g0 + x;
+      int alo, ahi;
+      if (kPT > 0) {
+        alo = (4 * g) < kPT ? 0 : ((4 * g) < kPT + kPH ? 1 : 2);
+        ahi = (4 * g + 3) < kPT ? 0 : ((4 * g + 3) < kPT + kPH ? 1 : 2);
+      } else {
+        alo = p.ch_ax_lo[g];
+        ahi = p.ch_ax_hi[g];
       }
-      *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      addr[x] = row_addr + uint32_t(g >> 3) * kHalfBytes + ((uint32_t(g & 7) ^ swz) << 4);
+      v[x] = ptx::lds128(addr[x]);
+      const uint32_t e_lo = uint32_t(p.ch_base_lo[g] + pick3(alo, pt, ph, pw)) * 16u;
+      C[x] = ptx::lds128f(tabC + e_lo);
+      S[x] = ptx::lds128f(tabS + e_lo);
+      if (alo != ahi) {
+        const uint32_t e_hi = uint32_t(p.ch_base_hi[g] + pick3(ahi, pt, ph, pw)) * 16u;
+        const float4 C2 = ptx::lds128f(tabC + e_hi);
+        const float4 S2 = ptx::lds128f(tabS + e_hi);
+        C[x] = make_float4(C[x].x * C2.x, C[x].y * C2.y, C[x].z * C2.z, C[x].w * C2.w);
+        S[x] = make_float4(S[x].x + S2.x, S[x].y + S2.y, S[x].z + S2.z, S[x].w + S2.w);
+      }
     }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) ptx::sts128(addr[x], rotate_chunk(v[x], C[x], S[x]));
   }
 }
 
-// Row max of one S tile (raw scores); columns >= lim are hidden when MASKED.
-template <bool MASKED>
-__device__ __forceinline__ float tile_rowmax(uint32_t tS, int lim) {
-  uint32_t r[32];
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    ptx::tmem_ld32(tS + ch * 32, r);
-    ptx::tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float v = __uint_as_float(r[i]);
-      if (MASKED && ch * 32 + i >= lim) v = -INFINITY;
-      mx[i & 3] = fmaxf(mx[i & 3], v);
-    }
-  }
-  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-}
-
-// P = exp2(S*scale_log2 - m) as bf16 into the first 64 columns of the S
-// region (P of columns 32c.. goes to packed columns 16c.., which the loop has
-// already read); returns the row sum of the fp32 P values.
-template <bool MASKED>
-__device__ __forceinline__ float tile_exp_store(uint32_t tS, int lim, float scale_log2, float m_use) {
-  uint32_t r[32];
-  float acc[2] = {0.f, 0.f};
-#pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    ptx::tmem_ld32(tS + ch * 32, r);
-    ptx::tmem_wait_ld();
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float p0 = ptx::ex2_approx(fmaf(__uint_as_float(r[2 * i]), scale_log2, -m_use));
-      float p1 = ptx::ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), scale_log2, -m_use));
-      if (MASKED && ch * 32 + 2 * i >= lim) p0 = 0.f;
-      if (MASKED && ch * 32 + 2 * i + 1 >= lim) p1 = 0.f;
-      acc[i & 1] += p0 + p1;
-      pk[i] = pack_bf16x2(p0, p1);
-    }
-    ptx::tmem_st16(tS + ch * 16, pk);
-  }
-  return acc[0] + acc[1];
+// Three-input max (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
@@ -262,6 +290,18 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk) {
   return ptx::smem_desc_sw128(tile + uint32_t(kk) * 2048u, kHalfBytes, 1024);
 }
 
+__device__ __forceinline__ void setmaxnreg_inc_softmax() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+}
+__device__ __forceinline__ void setmaxnreg_dec_rope() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegRope));
+}
+__device__ __forceinline__ void setmaxnreg_dec_producer() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
+}
+
+// kPT/kPH: compile-time RoPE axis split (pairs on t and h), or 0/0 for any split
+template <int kPT, int kPH>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -272,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8);
   int* abort_flag = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 4);
-  float2* tab = reinterpret_cast<float2*>(smem + kOffTab);
+  uint8_t* tab = smem + kOffTab;
   Ctx c;
   c.bar0 = sbase + kOffBar;
   c.abort = abort_flag;
@@ -305,20 +345,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
   // cos/sin table (fp64 sincos rounded to fp32) for every reachable position
   for (int e = tid; e < p.tab_entries; e += kThreads) {
-    int pos, i, n;
-    if (e < p.tab_base_h) {
-      const int ft = e / p.pt;
-      i = e - ft * p.pt; n = p.pt; pos = p.t_lo + ft;
-    } else if (e < p.tab_base_w) {
-      const int hh = (e - p.tab_base_h) / p.ph;
-      i = (e - p.tab_base_h) - hh * p.ph; n = p.ph; pos = hh;
-    } else {
-      const int ww = (e - p.tab_base_w) / p.pw;
-      i = (e - p.tab_base_w) - ww * p.pw; n = p.pw; pos = ww;
+    const int a = e < p.ax_tab[1] ? 0 : (e < p.ax_tab[2] ? 1 : 2);
+    const int rel = e - p.ax_tab[a];
+    const int k = rel / p.ax_npos[a];
+    const int pos_i = rel - k * p.ax_npos[a];
+    const int chunk = p.ax_chunk0[a] + k;
+    const int pos = a == 0 ? p.t_lo + pos_i : pos_i;
+    float cs[4], sn[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = 4 * chunk + j - p.ax_first[a];
+      double sd = 0.0, cd = 1.0;
+      if (i >= 0 && i < p.ax_count[a])
+        sincos(double(pos) * exp2(-(double(i) / double(p.ax_count[a])) * p.log2_theta), &sd, &cd);
+      cs[j] = __double2float_rn(cd);
+      sn[j] = __double2float_rn(sd);
     }
-    double s, co;
-    sincos(double(pos) * exp2(-(double(i) / double(n)) * p.log2_theta), &s, &co);
-    tab[e] = make_float2(__double2float_rn(co), __double2float_rn(s));
+    *reinterpret_cast<float4*>(tab + e * 16) = make_float4(cs[0], cs[1], cs[2], cs[3]);
+    *reinterpret_cast<float4*>(tab + (p.tab_entries + e) * 16) = make_float4(sn[0], sn[1], sn[2], sn[3]);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -326,9 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t tmem_base = *tmem_slot;
 
   const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV;
+  const uint32_t sTabC = sbase + kOffTab, sTabS = sTabC + uint32_t(p.tab_entries) * 16u;
 
   if (warp < 8) {
     // ===================== softmax (two warpgroups) =====================
+    setmaxnreg_inc_softmax();
     const int wg = warp >> 2;
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem_base + lane_off + col_s(wg);
@@ -344,33 +390,68 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int j = 0; j < un.nkt; ++j, ++g) {
         if (!wait_warp(c, bar(c, B_SFULL + wg), g & 1u, 1)) goto done;
         ptx::tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) ptx::tmem_ld32(tS + ch * 32, sr[ch]);
+        ptx::tmem_wait_ld();
         const int64_t kbase = int64_t(j) * kBN;
         const int lim = kbase + kBN > my_limit ? int(my_limit - kbase) : kBN;
         const bool masked = __any_sync(0xffffffffu, lim < kBN);
-        const float mx = masked ? tile_rowmax<true>(tS, lim) : tile_rowmax<false>(tS, lim);
+        if (masked) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], __uint_as_float(sr[ch][i]), __uint_as_float(sr[ch][i + 1]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m, mx * scale_log2);
         const bool need = m_new > m + kRescaleLog2;
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O holds tiles 0..j-1: wait for the last PV, then rescale in TMEM
-          if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 2)) goto done;
-          ptx::tc_fence_after();
-          const float f = need ? ptx::ex2_approx(m - m_new) : 1.0f;
-          uint32_t r[32];
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            ptx::tmem_ld32(tO + ch * 32, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            ptx::tmem_st32(tO + ch * 32, r);
-          }
-          ptx::tmem_wait_st();
-          l *= f;
-        }
+        const float m_old = m;
         if (need) m = m_new;
         const float m_use = (m == -INFINITY) ? 0.f : m;
-        l += masked ? tile_exp_store<true>(tS, lim, scale_log2, m_use)
-                    : tile_exp_store<false>(tS, lim, scale_log2, m_use);
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        const float2 nm2 = make_float2(-m_use, -m_use);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[ch][2 * i]), __uint_as_float(sr[ch][2 * i + 1])),
+                                        sc2, nm2);
+            const float2 pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));  // masked: exp2(-inf) = 0
+            acc[i & 3] = __fadd2_rn(acc[i & 3], pp);
+            pk[i] = pack_bf16x2(pp.x, pp.y);
+          }
+          ptx::tmem_st16(tS + ch * 16, pk);   // P (bf16) overwrites S columns 0..63
+        }
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+        const float tile_sum = (a01.x + a01.y) + (a23.x + a23.y);
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds tiles 0..j-1 scaled to the old max: wait for the last PV,
+          // then rescale in TMEM (PV(j) is not issued before P_FULL below)
+          if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 2)) goto done;
+          ptx::tc_fence_after();
+          const float f = need ? ptx::ex2_approx(m_old - m_new) : 1.0f;
+#pragma unroll 1
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t r[16];
+            ptx::tmem_ld16(tO + ch * 16, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+            ptx::tmem_st16(tO + ch * 16, r);
+          }
+          l *= f;
+        }
+        l += tile_sum;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(c, B_PFULL + wg));
@@ -380,17 +461,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       ptx::tc_fence_after();
       {
         const float inv = l > 0.f ? 1.0f / l : 0.f;
-        uint32_t r[32];
         uint8_t* orow = s.o + int64_t(qrow) * s.o_stride_bytes + int64_t(un.head) * (kHD * 2);
+        uint32_t r[4][32];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          ptx::tmem_ld32(tO + ch * 32, r);
-          ptx::tmem_wait_ld();
-          uint32_t pk[16];
+        for (int ch = 0; ch < 4; ++ch) ptx::tmem_ld32(tO + ch * 32, r[ch]);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(c, B_OFREE + wg));   // O may now be overwritten
+        if (qrow < s.Lq) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-          if (qrow < s.Lq) {
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(r[ch][2 * i]) * inv, __uint_as_float(r[ch][2 * i + 1]) * inv);
             uint4* dst = reinterpret_cast<uint4*>(orow + ch * 64);
             dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -399,11 +483,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           }
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(c, B_OFREE + wg));
     }
   } else if (warp < 12) {
     // ===================== RoPE warpgroup =====================
+    setmaxnreg_dec_rope();
     const int rt = tid - 256;
     uint32_t it = 0, ul = 0;
     for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ul) {
@@ -412,21 +495,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (!wait_warp(c, bar(c, B_QFULL), ul & 1u, 4)) goto done;
       if (s.flags & RKV_ROPE_Q) {
         for (int b = 0; b < kSub; ++b)
-          rope_tile(p, tab, smem + kOffQ + b * kTileBytes, un.qb * kUnitRows + b * kBM, s.Lq, s.q_t0, rt);
+          rope_tile<kPT, kPH>(p, sTabC, sTabS, sQ + b * kTileBytes, un.qb * kUnitRows + b * kBM, s.Lq, s.q_t0, rt);
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(bar(c, B_QREADY));
       for (int j = 0; j < un.nkt; ++j, ++it) {
         const uint32_t st = it % kStages, n = it / kStages;
         if (!wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5)) goto done;
-        if (s.flags & RKV_ROPE_K) rope_tile(p, tab, smem + kOffK + st * kTileBytes, j * kBN, s.Lk, s.k_t0, rt);
+        if (s.flags & RKV_ROPE_K) rope_tile<kPT, kPH>(p, sTabC, sTabS, sK + st * kTileBytes, j * kBN, s.Lk, s.k_t0, rt);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(c, B_KREADY + st));
       }
     }
-  } else if (warp == 12) {
-    // ===================== TMA producer: Q and K =====================
-    if (lane == 0) {
+  } else {
+    setmaxnreg_dec_producer();
+    if (warp == 12 && lane == 0) {
+      // ===================== TMA producer: Q and K =====================
       for (int i = 0; i < p.n_seqs; ++i) {
         ptx::tma_prefetch_desc(&p.seq[i].tq);
         ptx::tma_prefetch_desc(&p.seq[i].tk);
@@ -452,10 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         if (!ok) break;
       }
-    }
-  } else if (warp == 14) {
-    // ===================== TMA producer: V =====================
-    if (lane == 0) {
+    } else if (warp == 14 && lane == 0) {
+      // ===================== TMA producer: V =====================
       for (int i = 0; i < p.n_seqs; ++i) ptx::tma_prefetch_desc(&p.seq[i].tv);
       uint32_t it = 0;
       bool ok = true;
@@ -471,10 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                              j * kBN);
         }
       }
-    }
-  } else if (warp == 13) {
-    // ===================== MMA issuer =====================
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ===================== MMA issuer =====================
       const uint32_t id_s = ptx::idesc_bf16_f32(kBM, kBN, false);
       const uint32_t id_pv = ptx::idesc_bf16_f32(kBM, kHD, true);
       uint32_t it = 0, g = 0, ul = 0;
@@ -698,18 +778,43 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   if (units >= (int64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "too many work units");
   if (t_lo == INT64_MAX) { t_lo = 0; t_hi = -1; }
   const int64_t n_t = t_hi - t_lo + 1;
-  const int64_t entries = n_t * rope->pairs_t + int64_t(rope->grid_h) * rope->pairs_h + int64_t(rope->grid_w) * rope->pairs_w;
-  if (entries > kMaxTab)
-    return fail(RKV_ERR_UNSUPPORTED, "RoPE positions need %lld cos/sin entries (max %d)", (long long)entries, kMaxTab);
+  const int32_t pairs[3] = {rope->pairs_t, rope->pairs_h, rope->pairs_w};
+  for (int a = 0; a < 3; ++a)
+    if (pairs[a] < 4) return fail(RKV_ERR_UNSUPPORTED, "fused RoPE needs >= 4 rotary pairs per axis");
+  const int64_t npos[3] = {n_t, rope->grid_h, rope->grid_w};
+  int64_t entries = 0;
+  int32_t first = 0;
+  for (int a = 0; a < 3; ++a) {
+    p.ax_first[a] = first;
+    p.ax_count[a] = pairs[a];
+    p.ax_chunk0[a] = first / 4;
+    p.ax_nch[a] = (first + pairs[a] - 1) / 4 - first / 4 + 1;
+    p.ax_npos[a] = int32_t(std::max<int64_t>(npos[a], 1));
+    p.ax_tab[a] = int32_t(std::min<int64_t>(entries, INT32_MAX));
+    entries += int64_t(p.ax_npos[a]) * p.ax_nch[a];
+    first += pairs[a];
+  }
+  if (entries > kMaxTabEntries)
+    return fail(RKV_ERR_UNSUPPORTED, "RoPE positions need %lld cos/sin table entries (max %d)", (long long)entries,
+                kMaxTabEntries);
+  auto axis_of_pair = [&](int pr) { return pr < p.ax_first[1] ? 0 : (pr < p.ax_first[2] ? 1 : 2); };
+  for (int g = 0; g < 16; ++g) {
+    const int alo = axis_of_pair(4 * g), ahi = axis_of_pair(4 * g + 3);
+    p.ch_ax_lo[g] = int8_t(alo);
+    p.ch_ax_hi[g] = int8_t(ahi);
+    p.ch_base_lo[g] = p.ax_tab[alo] + (g - p.ax_chunk0[alo]) * p.ax_npos[alo];
+    p.ch_base_hi[g] = p.ax_tab[ahi] + (g - p.ax_chunk0[ahi]) * p.ax_npos[ahi];
+    int sel = 0;
+    if (ahi != alo)
+      for (int j = 0; j < 4; ++j) sel |= (axis_of_pair(4 * g + j) == ahi) << j;
+    p.ch_sel[g] = int8_t(sel);
+  }
   p.n_seqs = n_seqs;
   p.H = H;
   p.total_units = int32_t(units);
   p.scale_log2 = float(double(softmax_scale) * 1.4426950408889634);
   p.grid_h = rope->grid_h; p.grid_w = rope->grid_w;
-  p.pt = rope->pairs_t; p.ph = rope->pairs_h; p.pw = rope->pairs_w;
   p.t_lo = int32_t(t_lo); p.n_t = int32_t(n_t);
-  p.tab_base_h = int32_t(n_t * rope->pairs_t);
-  p.tab_base_w = p.tab_base_h + rope->grid_h * rope->pairs_h;
   p.tab_entries = int32_t(entries);
   p.F = uint32_t(F);
   p.div_F = make_fastdiv(uint32_t(F));
@@ -721,10 +826,13 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWorkspaceBytes, cs);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
-  e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  // the 22/21/21 split of the pages' 128-dim heads gets its own instantiation
+  const bool default_split = rope->pairs_t == 22 && rope->pairs_h == 21 && rope->pairs_w == 21;
+  auto kern = default_split ? attn_fwd_kernel<22, 21> : attn_fwd_kernel<0, 0>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
   const int grid = int(std::min<int64_t>(units, sm_count()));
-  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, cs>>>(p);
+  kern<<<grid, kThreads, kSmemBytes, cs>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return RKV_OK;

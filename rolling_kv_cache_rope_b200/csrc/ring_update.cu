@@ -139,7 +139,7 @@ extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, con
     a.div_F = make_fastdiv(a.F);
     const uint64_t per_block = uint64_t(kRingThreads) * kRingUnroll;
     uint64_t blocks = (total_vecs + per_block - 1) / per_block;
-    const uint64_t wave = uint64_t(sm_count()) * (2048 / kRingThreads) / 2;  // two tensors share the wave
+    const uint64_t wave = uint64_t(sm_count()) * (2048 / kRingThreads);  // per tensor: two resident waves in all
     if (blocks > wave) blocks = wave;
     dim3 grid(uint32_t(blocks), 2);
     ring_copy_kernel<<<grid, kRingThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
