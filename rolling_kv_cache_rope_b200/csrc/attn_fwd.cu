@@ -42,6 +42,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "exp2_fma.cuh"
 #include "sm100_ptx.cuh"
 
 namespace rkv {
@@ -61,9 +62,12 @@ constexpr int kThreads = 16 * 32;
 constexpr int kTabEntryBytes = 32;   // cos and sin of 4 consecutive rotary pairs
 constexpr int kMaxTabEntries = 768;  // 24 KB of shared memory (cos array, then sin array)
 constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growth
+// Route one exponential pair in four to the FMA pipe.  Off: measured slower
+// on B200 at this kernel's operating point (the softmax is not MUFU-bound).
+constexpr bool kPolyExp = false;
 // register split (setmaxnreg): two softmax warpgroups, RoPE, producers; the
 // four shares add up to the 4 x 128 registers per thread the block launches with
-constexpr int kRegSoftmax = 168, kRegRope = 96, kRegProducer = 80;
+constexpr int kRegSoftmax = 168, kRegRope = 88, kRegProducer = 88;
 static_assert(2 * kRegSoftmax + kRegRope + kRegProducer == 4 * 128, "register split must match the launch");
 
 // shared-memory map (offsets from a 1024-byte aligned base)
@@ -283,6 +287,37 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
+// P = exp2(S * scale_log2 - m_use) for one thread's row of S (in registers),
+// written as bf16 over the first 64 TMEM columns of the S region; returns the
+// row sum of the fp32 P.  kPoly: one pair in four takes the FMA-pipe exp2 (not
+// in masked tiles, whose hidden scores are -inf).
+template <bool kPoly>
+__device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uint32_t tS, float scale_log2,
+                                                float m_use) {
+  const float2 sc2 = make_float2(scale_log2, scale_log2);
+  const float2 nm2 = make_float2(-m_use, -m_use);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 x =
+          __ffma2_rn(make_float2(__uint_as_float(sr[ch][2 * i]), __uint_as_float(sr[ch][2 * i + 1])), sc2, nm2);
+      float2 pp;
+      if (kPoly && (i & 3) == 3)
+        pp = rkv::exp2_fma2(x);
+      else
+        pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));  // exp2(-inf) = 0 for hidden keys
+      acc[i & 3] = __fadd2_rn(acc[i & 3], pp);
+      pk[i] = pack_bf16x2(pp.x, pp.y);
+    }
+    ptx::tmem_st16(tS + ch * 16, pk);   // P (bf16) overwrites S columns 0..63
+  }
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  return (a01.x + a01.y) + (a23.x + a23.y);
+}
+
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
   return ptx::smem_desc_sw128(tile + uint32_t(kk >> 2) * kHalfBytes + uint32_t(kk & 3) * 32u, 16, 1024);
 }
@@ -416,24 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const float m_old = m;
         if (need) m = m_new;
         const float m_use = (m == -INFINITY) ? 0.f : m;
-        const float2 sc2 = make_float2(scale_log2, scale_log2);
-        const float2 nm2 = make_float2(-m_use, -m_use);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[ch][2 * i]), __uint_as_float(sr[ch][2 * i + 1])),
-                                        sc2, nm2);
-            const float2 pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));  // masked: exp2(-inf) = 0
-            acc[i & 3] = __fadd2_rn(acc[i & 3], pp);
-            pk[i] = pack_bf16x2(pp.x, pp.y);
-          }
-          ptx::tmem_st16(tS + ch * 16, pk);   // P (bf16) overwrites S columns 0..63
-        }
-        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-        const float tile_sum = (a01.x + a01.y) + (a23.x + a23.y);
+        const float tile_sum = masked ? exp_store_tile<false>(sr, tS, scale_log2, m_use)
+                                      : exp_store_tile<kPolyExp>(sr, tS, scale_log2, m_use);
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O holds tiles 0..j-1 scaled to the old max: wait for the last PV,
           // then rescale in TMEM (PV(j) is not issued before P_FULL below)
@@ -555,49 +574,57 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
     } else if (warp == 13 && lane == 0) {
       // ===================== MMA issuer =====================
+      // Waits on smem handoffs (Q/K after RoPE, V after TMA) need no tcgen05
+      // fence; waits on TMEM handoffs (P written with tcgen05.st, O read by
+      // the epilogue) do.  Descriptors are built once; a k-step only moves
+      // the 14-bit start-address field (addresses < 256 KB, so no carry).
       const uint32_t id_s = ptx::idesc_bf16_f32(kBM, kBN, false);
       const uint32_t id_pv = ptx::idesc_bf16_f32(kBM, kHD, true);
+      const uint64_t dq0 = desc_kmajor(sQ, 0), dq1 = desc_kmajor(sQ + kTileBytes, 0);
       uint32_t it = 0, g = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
         const Unit un = decode_unit(p, u);
         if (!wait_phase(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
-        ptx::tc_fence_after();
         for (int j = 0; j < un.nkt; ++j, ++it, ++g) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t kt = sK + st * kTileBytes;
+          const uint64_t dk = desc_kmajor(sK + st * kTileBytes, 0);
           if (j > 0) {
             const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
             if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 11)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const uint32_t vt = sV + sp * kTileBytes;
+            const uint64_t dv = desc_v(sV + sp * kTileBytes, 0);
             for (int b = 0; b < kSub && ok; ++b) {
               if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 12)) { ok = false; break; }
-              ptx::tc_fence_after();
               if (j == 1) {
                 if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 13)) { ok = false; break; }
-                ptx::tc_fence_after();
               }
+              ptx::tc_fence_after();
               // O_b (+)= P_b(j-1) V(j-1): P from TMEM, V from shared memory (MN-major)
+#pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, desc_v(vt, kk), id_pv,
-                            (j > 1 || kk > 0) ? 1u : 0u);
+                ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)),
+                            id_pv, (j > 1 || kk > 0) ? 1u : 0u);
               ptx::mma_commit(bar(c, B_ODONE + b));
               // S_b(j) = Q_b K(j)^T
-              const uint32_t qt = sQ + b * kTileBytes;
-              for (int kk = 0; kk < 8; ++kk)
-                ptx::mma_ss(tmem_base + col_s(b), desc_kmajor(qt, kk), desc_kmajor(kt, kk), id_s, kk > 0 ? 1u : 0u);
+              const uint64_t dq = b ? dq1 : dq0;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t off = uint64_t(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+                ptx::mma_ss(tmem_base + col_s(b), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
+              }
               ptx::mma_commit(bar(c, B_SFULL + b));
             }
             if (!ok) break;
             ptx::mma_commit(bar(c, B_VFREE + sp));
           } else {
             for (int b = 0; b < kSub; ++b) {
-              const uint32_t qt = sQ + b * kTileBytes;
-              for (int kk = 0; kk < 8; ++kk)
-                ptx::mma_ss(tmem_base + col_s(b), desc_kmajor(qt, kk), desc_kmajor(kt, kk), id_s, kk > 0 ? 1u : 0u);
+              const uint64_t dq = b ? dq1 : dq0;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t off = uint64_t(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+                ptx::mma_ss(tmem_base + col_s(b), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
+              }
               ptx::mma_commit(bar(c, B_SFULL + b));
             }
           }
@@ -608,17 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // PV of the unit's last tile
         const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
         if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 14)) { ok = false; break; }
-        ptx::tc_fence_after();
-        const uint32_t vt = sV + sp * kTileBytes;
+        const uint64_t dv = desc_v(sV + sp * kTileBytes, 0);
         for (int b = 0; b < kSub && ok; ++b) {
           if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 15)) { ok = false; break; }
-          ptx::tc_fence_after();
           if (un.nkt == 1) {
             if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 16)) { ok = false; break; }
-            ptx::tc_fence_after();
           }
+          ptx::tc_fence_after();
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, desc_v(vt, kk), id_pv,
+            ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)), id_pv,
                         (un.nkt > 1 || kk > 0) ? 1u : 0u);
           ptx::mma_commit(bar(c, B_ODONE + b));
         }
