@@ -13,24 +13,33 @@
 // ("Optimizing Real-Time Video Generation on Trainium Chips", item 8 "Model
 // structure optimizations").
 //
-// Design (one CTA per SM, 15 warps):
+// Design: clusters of two CTAs on two SMs share every MMA (tcgen05
+// cta_group::2, M = 256 query rows), 16 warps per CTA:
 //   warps 0-3   softmax for Q sub-tile 0 (one TMEM lane = one query row each)
 //   warps 4-7   softmax for Q sub-tile 1
-//   warps 8-11  RoPE: rotate the Q sub-tiles and each K tile in shared memory
-//               right after TMA lands them, before the tensor core reads them
+//   warps 8-11  RoPE: rotate this CTA's Q rows and its half of each K tile in
+//               shared memory right after TMA lands them
 //   warp 12     TMA producer for Q and K;  warp 14  TMA producer for V
-//   warp 13     allocates TMEM; one lane issues every tcgen05.mma
-// A work unit is (sequence, head, 256 query rows).  Q/K/V are read straight
-// from token-major [L][H][128] tensors through 3-D TMA descriptors (head is a
-// coordinate), so no transpose pass exists.  S = Q K^T (128x128 fp32) and the
-// running O (128x128 fp32) of both sub-tiles live in TMEM (4 x 128 columns).
-// Softmax reads S with tcgen05.ld, writes P as bf16 back into the first 64
-// columns of the same S region, and the PV MMA takes P straight from TMEM.
-// While one softmax warpgroup works, the tensor core runs the other
-// sub-tile's MMAs (ping-pong).  The running max is only moved (and O rescaled
-// in TMEM) when it grows by more than 2^8, which after the first tile almost
-// never happens.  All waits are bounded; a stuck wait makes every role stop,
-// records RKV_ERR_TIMEOUT in the workspace and frees TMEM.
+//   warp 13     allocates TMEM (both CTAs); in the leader CTA one lane issues
+//               every tcgen05.mma for the pair
+//   warp 15     tells the leader when this CTA's V half has landed
+// A work unit is (sequence, head, 512 query rows); each CTA owns 256 rows as
+// two 128-row sub-tiles.  A 2-CTA MMA splits its B operand by N between the
+// two CTAs, so each CTA loads and rotates only 64 keys of every 128-key K tile
+// and only 64 of the 128 columns of every V tile: shared-memory traffic per SM
+// (operand reads, TMA writes, RoPE) halves against a one-CTA MMA, which is
+// what bounds a 128x128 tile on one SM.  Q/K/V are read straight from
+// token-major [L][H][128] tensors through 3-D TMA descriptors (head is a
+// coordinate), so no transpose pass exists.  S = Q K^T (128x128 fp32 per CTA)
+// and the running O of both sub-tiles live in TMEM (4 x 128 columns).
+// Softmax reads S with tcgen05.ld, writes P as bf16 over the first 64 columns
+// of the same S region, and the PV MMA takes P straight from TMEM.  While one
+// softmax warpgroup works, the tensor cores run the other sub-tile's MMAs
+// (ping-pong).  The running max is only moved (and O rescaled in TMEM) when it
+// grows by more than 2^8.  Operand readiness is reported to the leader with
+// cluster-scope mbarrier arrives; the leader's commits are multicast to both
+// CTAs.  No TMA load uses multicast.  All waits are bounded: a stuck wait makes
+// the CTA stop, records RKV_ERR_TIMEOUT in the workspace and frees TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -51,13 +60,18 @@ rkv_status check_rope(const rkv_rope3d* rope, int32_t D);
 namespace attn {
 
 constexpr int kBM = 128;             // query rows per sub-tile (one TMEM lane each)
-constexpr int kSub = 2;              // sub-tiles per unit
-constexpr int kUnitRows = kBM * kSub;
-constexpr int kBN = 128;             // keys per K/V tile
+constexpr int kSub = 2;              // sub-tiles per CTA
+constexpr int kCtaRows = kBM * kSub; // 256 query rows per CTA
+constexpr int kUnitRows = 2 * kCtaRows;   // 512 query rows per CTA pair
+constexpr int kBN = 128;             // keys per K/V tile (per pair)
 constexpr int kHD = 128;             // head dim
-constexpr int kStages = 2;           // K and V pipeline depth
-constexpr int kTileBytes = kBN * kHD * 2;      // 32 KB
-constexpr int kHalfBytes = kTileBytes / 2;     // 128 rows x 64 cols
+constexpr int kStages = 4;           // K and V pipeline depth
+constexpr int kQTileBytes = kBM * kHD * 2;     // 32 KB: 128 rows x 128 cols
+constexpr int kQHalfBytes = kQTileBytes / 2;   // 128 rows x 64 cols
+constexpr int kKRows = kBN / 2;                // keys of a K tile held by one CTA
+constexpr int kKStageBytes = kKRows * kHD * 2; // 16 KB: 64 rows x 128 cols
+constexpr int kKHalfBytes = kKStageBytes / 2;  // 64 rows x 64 cols
+constexpr int kVStageBytes = kBN * 64 * 2;     // 16 KB: 128 rows x 64 cols
 constexpr int kThreads = 16 * 32;
 constexpr int kTabEntryBytes = 32;   // cos and sin of 4 consecutive rotary pairs
 constexpr int kMaxTabEntries = 768;  // 24 KB of shared memory (cos array, then sin array)
@@ -67,16 +81,17 @@ constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growt
 constexpr bool kPolyExp = false;
 // register split (setmaxnreg): two softmax warpgroups, RoPE, producers; the
 // four shares add up to the 4 x 128 registers per thread the block launches with
-constexpr int kRegSoftmax = 168, kRegRope = 88, kRegProducer = 88;
+constexpr int kRegSoftmax = 176, kRegRope = 80, kRegProducer = 80;
 static_assert(2 * kRegSoftmax + kRegRope + kRegProducer == 4 * 128, "register split must match the launch");
 
-// shared-memory map (offsets from a 1024-byte aligned base)
+// shared-memory map (offsets from a 1024-byte aligned base; identical in both CTAs)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kSub * kTileBytes;
-constexpr int kOffV = kOffK + kStages * kTileBytes;
-constexpr int kOffTab = kOffV + kStages * kTileBytes;
+constexpr int kOffK = kOffQ + kSub * kQTileBytes;
+constexpr int kOffV = kOffK + kStages * kKStageBytes;
+constexpr int kOffTab = kOffV + kStages * kVStageBytes;
 constexpr int kOffBar = kOffTab + kMaxTabEntries * kTabEntryBytes;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;   // + alignment slack
+constexpr int kBarBytes = 512;
+constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
 
 // TMEM columns: S of sub-tile b at 128*b, O of sub-tile b at 256 + 128*b
 __host__ __device__ constexpr uint32_t col_s(int b) { return 128u * uint32_t(b); }
@@ -117,15 +132,17 @@ struct Params {
   uint64_t timeout_ns;
 };
 
-// barrier indices
+// barrier indices.  The first group is used in every CTA; the second only in
+// the leader (rank 0), where both CTAs arrive on it.
 enum : int {
-  B_QFULL = 0, B_QREADY, B_QFREE,
-  B_KFULL, B_KREADY = B_KFULL + kStages, B_KFREE = B_KREADY + kStages,
+  B_QFULL = 0, B_QFREE,
+  B_KFULL, B_KFREE = B_KFULL + kStages,
   B_VFULL = B_KFREE + kStages, B_VFREE = B_VFULL + kStages,
-  B_SFULL = B_VFREE + kStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_OFREE = B_ODONE + 2,
-  B_FINAL = B_OFREE + 2, B_COUNT
+  B_SFULL = B_VFREE + kStages, B_ODONE = B_SFULL + 2, B_FINAL = B_ODONE + 2,
+  B_QREADY, B_KREADY, B_VREADY = B_KREADY + kStages, B_PFULL = B_VREADY + kStages, B_OFREE = B_PFULL + 2,
+  B_COUNT = B_OFREE + 2
 };
-static_assert(B_COUNT * 8 + 16 <= 256, "barrier area");
+static_assert(B_COUNT * 8 + 16 <= kBarBytes, "barrier area");
 
 struct Ctx {
   uint32_t bar0;         // shared address of barrier 0
@@ -155,6 +172,13 @@ __device__ __forceinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t pa
   }
 }
 
+// The same for a barrier that the peer CTA also arrives on.  The handoffs
+// through such barriers carry TMEM or async-proxy shared-memory data, ordered
+// by tcgen05 / proxy fences, so the wait keeps the default (CTA) scope.
+__device__ __forceinline__ bool wait_phase_cluster(const Ctx& c, uint32_t b, uint32_t parity, int where) {
+  return wait_phase(c, b, parity, where);
+}
+
 // Warp-uniform variant for roles whose 32 lanes continue together.
 __device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t b, uint32_t parity, int where) {
   const bool ok = wait_phase(c, b, parity, where);
@@ -173,10 +197,10 @@ __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p
   return lim < s.Lk ? lim : s.Lk;
 }
 
-// Units are numbered head-major within a sequence (all query blocks of head 0,
-// then head 1, ...), so the CTAs in flight at any time share the K/V tiles of
-// one or two heads in L2.  Masked sequences list their query blocks from the
-// most to the least visible keys.
+// Units (512 query rows, one per CTA pair) are numbered head-major within a
+// sequence (all query blocks of head 0, then head 1, ...), so the clusters in
+// flight at any time share the K/V tiles of one or two heads in L2.  Masked
+// sequences list their query blocks from the most to the least visible keys.
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   Unit r;
   int si = 0;
@@ -221,12 +245,12 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 v, float4 C, float4 S) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// RoPE of one 128-row tile in shared memory (128B-swizzled, 2 halves), in
-// place.  Thread rt owns row rt: its (t, h, w) is computed once and it walks
-// the row's 16 chunks (4 rotary pairs each).  Chunk g lies on the same axis
-// for every thread, so all branches are warp-uniform, and neighbouring rows
-// read broadcast (t, h) or adjacent (w) table entries.  Loads for 4 chunks
-// are issued before their arithmetic.
+// RoPE of one row (chunks [kG0, kG0 + kGN) of its 16) of a 128B-swizzled
+// tile in shared memory, in place.  `row_addr` is the row's address in the
+// tile's first 64-column half, `half_stride` the distance to the second half.
+// Chunk g lies on the same axis for every thread of a warp, so branches are
+// warp-uniform, and neighbouring rows read broadcast (t, h) or adjacent (w)
+// table entries.  Loads for 4 chunks are issued before their arithmetic.
 //
 // A chunk that straddles two axes reads both axes' entries; each axis' table
 // holds cos 1 / sin 0 for pairs outside the axis, so the chunk's cos and sin
@@ -235,19 +259,11 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 v, float4 C, float4 S) {
 // kPT/kPH > 0: the axis split is known at compile time (chunk -> axis folds to
 // constants and only straddling chunks load twice); kPT == 0: read it from
 // the parameters.
-template <int kPT, int kPH>
-__device__ __forceinline__ void rope_tile(const Params& p, uint32_t tabC, uint32_t tabS, uint32_t tile, int row0,
-                                          int limit, int t0, int rt) {
-  const int row = row0 + rt;
-  if (row >= limit) return;
-  const uint32_t f = fdiv(uint32_t(row), p.div_F);
-  const uint32_t in_f = uint32_t(row) - f * p.F;
-  const uint32_t hh = fdiv(in_f, p.div_W);
-  const int pt = t0 + int(f) - p.t_lo, ph = int(hh), pw = int(in_f - hh * uint32_t(p.grid_w));
-  const uint32_t row_addr = tile + uint32_t(rt) * 128u;
-  const uint32_t swz = uint32_t(rt & 7);
+template <int kPT, int kPH, int kG0, int kGN>
+__device__ __forceinline__ void rope_row(const Params& p, uint32_t tabC, uint32_t tabS, uint32_t row_addr,
+                                         uint32_t half_stride, uint32_t swz, int pt, int ph, int pw) {
 #pragma unroll
-  for (int g0 = 0; g0 < 16; g0 += 4) {
+  for (int g0 = kG0; g0 < kG0 + kGN; g0 += 4) {
     uint4 v[4];
     float4 C[4], S[4];
     uint32_t addr[4];
@@ -262,7 +278,7 @@ __device__ __forceinline__ void rope_tile(const Params& p, uint32_t tabC, uint32
         alo = p.ch_ax_lo[g];
         ahi = p.ch_ax_hi[g];
       }
-      addr[x] = row_addr + uint32_t(g >> 3) * kHalfBytes + ((uint32_t(g & 7) ^ swz) << 4);
+      addr[x] = row_addr + uint32_t(g >> 3) * half_stride + ((uint32_t(g & 7) ^ swz) << 4);
       v[x] = ptx::lds128(addr[x]);
       const uint32_t e_lo = uint32_t(p.ch_base_lo[g] + pick3(alo, pt, ph, pw)) * 16u;
       C[x] = ptx::lds128f(tabC + e_lo);
@@ -278,6 +294,16 @@ __device__ __forceinline__ void rope_tile(const Params& p, uint32_t tabC, uint32
 #pragma unroll
     for (int x = 0; x < 4; ++x) ptx::sts128(addr[x], rotate_chunk(v[x], C[x], S[x]));
   }
+}
+
+// (t, h, w) table positions of token `row` of a sequence whose first frame is t0.
+__device__ __forceinline__ void row_positions(const Params& p, int row, int t0, int& pt, int& ph, int& pw) {
+  const uint32_t f = fdiv(uint32_t(row), p.div_F);
+  const uint32_t in_f = uint32_t(row) - f * p.F;
+  const uint32_t hh = fdiv(in_f, p.div_W);
+  pt = t0 + int(f) - p.t_lo;
+  ph = int(hh);
+  pw = int(in_f - hh * uint32_t(p.grid_w));
 }
 
 // Three-input max (sm_100).
@@ -318,12 +344,16 @@ __device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uin
   return (a01.x + a01.y) + (a23.x + a23.y);
 }
 
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
-  return ptx::smem_desc_sw128(tile + uint32_t(kk >> 2) * kHalfBytes + uint32_t(kk & 3) * 32u, 16, 1024);
+// K-major operand (rows of 128 bf16 in two 64-column 128B-swizzled halves):
+// 8-row groups 1024 bytes apart; k-step kk starts 32 bytes further inside a
+// half, or in the second half from kk = 4.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile) { return ptx::smem_desc_sw128(tile, 16, 1024); }
+__device__ __forceinline__ uint64_t kstep_off(int kk, int half_bytes) {
+  return uint64_t(((kk >> 2) * half_bytes + (kk & 3) * 32) >> 4);
 }
-__device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk) {
-  return ptx::smem_desc_sw128(tile + uint32_t(kk) * 2048u, kHalfBytes, 1024);
-}
+// V half (128 keys x 64 columns, 128B-swizzled) as the MN-major B operand of
+// PV: keys are K, 8-key groups 1024 bytes apart; k-step kk = 16 keys = 2048 B.
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile) { return ptx::smem_desc_sw128(tile, kVStageBytes, 1024); }
 
 __device__ __forceinline__ void setmaxnreg_inc_softmax() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
@@ -344,6 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const uint32_t rank = ptx::cluster_ctarank();   // 0 = leader of the pair
+  const int cluster = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8);
   int* abort_flag = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 4);
@@ -352,31 +385,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   c.bar0 = sbase + kOffBar;
   c.abort = abort_flag;
   c.p = &p;
+  // a leader-side barrier, addressed from either CTA
+  auto lbar = [&](int i) { return ptx::mapa_shared(bar(c, i), 0); };
 
   if (tid == 0) {
     ptx::mbar_init(bar(c, B_QFULL), 1);
-    ptx::mbar_init(bar(c, B_QREADY), 128);
     ptx::mbar_init(bar(c, B_QFREE), 1);
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(bar(c, B_KFULL + s), 1);
-      ptx::mbar_init(bar(c, B_KREADY + s), 128);
       ptx::mbar_init(bar(c, B_KFREE + s), 1);
       ptx::mbar_init(bar(c, B_VFULL + s), 1);
       ptx::mbar_init(bar(c, B_VFREE + s), 1);
+      ptx::mbar_init(bar(c, B_KREADY + s), 2);      // one arrive per CTA
+      ptx::mbar_init(bar(c, B_VREADY + s), 2);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(c, B_SFULL + b), 1);
-      ptx::mbar_init(bar(c, B_PFULL + b), 128);
       ptx::mbar_init(bar(c, B_ODONE + b), 1);
-      ptx::mbar_init(bar(c, B_OFREE + b), 128);
+      ptx::mbar_init(bar(c, B_PFULL + b), 8);       // one arrive per softmax warp, both CTAs
+      ptx::mbar_init(bar(c, B_OFREE + b), 8);
     }
+    ptx::mbar_init(bar(c, B_QREADY), 2);
     ptx::mbar_init(bar(c, B_FINAL), 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 13) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc2(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish2();
   }
   // cos/sin table (fp64 sincos rounded to fp32) for every reachable position
   for (int e = tid; e < p.tab_entries; e += kThreads) {
@@ -401,6 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_arrive();   // both CTAs' barriers are initialised before any remote arrive
+  ptx::cluster_wait();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -414,12 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem_base + lane_off + col_s(wg);
     const uint32_t tO = tmem_base + lane_off + col_o(wg);
+    const uint32_t pfull = lbar(B_PFULL + wg), ofree = lbar(B_OFREE + wg);
     const float scale_log2 = p.scale_log2;
     uint32_t g = 0;
-    for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+    for (int u = cluster; u < p.total_units; u += n_clusters) {
       const Unit un = decode_unit(p, u);
       const SeqDev& s = p.seq[un.si];
-      const int qrow = un.qb * kUnitRows + wg * kBM + 32 * (warp & 3) + lane;
+      const int qrow = un.qb * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
       const int64_t my_limit = row_kv_limit(s, p, qrow < s.Lq ? qrow : s.Lq - 1);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < un.nkt; ++j, ++g) {
@@ -473,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         l += tile_sum;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(c, B_PFULL + wg));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(pfull);
       }
       // epilogue: O / l -> bf16 -> global (row-major [Lq][H][128])
       if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 3)) goto done;
@@ -486,7 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int ch = 0; ch < 4; ++ch) ptx::tmem_ld32(tO + ch * 32, r[ch]);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(c, B_OFREE + wg));   // O may now be overwritten
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(ofree);   // O may now be overwritten
         if (qrow < s.Lq) {
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -507,155 +548,195 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // ===================== RoPE warpgroup =====================
     setmaxnreg_dec_rope();
     const int rt = tid - 256;
+    const uint32_t qready = lbar(B_QREADY);
     uint32_t it = 0, ul = 0;
-    for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ul) {
+    for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
       const Unit un = decode_unit(p, u);
       const SeqDev& s = p.seq[un.si];
       if (!wait_warp(c, bar(c, B_QFULL), ul & 1u, 4)) goto done;
       if (s.flags & RKV_ROPE_Q) {
-        for (int b = 0; b < kSub; ++b)
-          rope_tile<kPT, kPH>(p, sTabC, sTabS, sQ + b * kTileBytes, un.qb * kUnitRows + b * kBM, s.Lq, s.q_t0, rt);
+        // thread rt rotates row rt of both Q sub-tiles (all 16 chunks)
+        for (int b = 0; b < kSub; ++b) {
+          const int row = un.qb * kUnitRows + int(rank) * kCtaRows + b * kBM + rt;
+          if (row < s.Lq) {
+            int pt, ph, pw;
+            row_positions(p, row, s.q_t0, pt, ph, pw);
+            rope_row<kPT, kPH, 0, 16>(p, sTabC, sTabS, sQ + uint32_t(b * kQTileBytes + rt * 128), kQHalfBytes,
+                                      uint32_t(rt & 7), pt, ph, pw);
+          }
+        }
       }
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar(c, B_QREADY));
+      ptx::named_sync(1, 128);
+      if (rt == 0) ptx::mbar_arrive_cluster(qready);
       for (int j = 0; j < un.nkt; ++j, ++it) {
         const uint32_t st = it % kStages, n = it / kStages;
         if (!wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5)) goto done;
-        if (s.flags & RKV_ROPE_K) rope_tile<kPT, kPH>(p, sTabC, sTabS, sK + st * kTileBytes, j * kBN, s.Lk, s.k_t0, rt);
+        if (s.flags & RKV_ROPE_K) {
+          // this CTA's 64 keys of the tile: two threads per key row, warps
+          // 8-9 take chunks 0-7 (first 64 columns), warps 10-11 chunks 8-15
+          const int r = rt & 63;
+          const int row = j * kBN + int(rank) * kKRows + r;
+          if (row < s.Lk) {
+            int pt, ph, pw;
+            row_positions(p, row, s.k_t0, pt, ph, pw);
+            const uint32_t ra = sK + st * kKStageBytes + uint32_t(r * 128);
+            if (rt < 64)
+              rope_row<kPT, kPH, 0, 8>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
+            else
+              rope_row<kPT, kPH, 8, 8>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
+          }
+        }
         ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(bar(c, B_KREADY + st));
+        ptx::named_sync(1, 128);
+        if (rt == 0) ptx::mbar_arrive_cluster(lbar(B_KREADY + st));
       }
     }
   } else {
     setmaxnreg_dec_producer();
     if (warp == 12 && lane == 0) {
-      // ===================== TMA producer: Q and K =====================
+      // ===================== TMA producer: Q and this CTA's K halves =====================
       for (int i = 0; i < p.n_seqs; ++i) {
         ptx::tma_prefetch_desc(&p.seq[i].tq);
         ptx::tma_prefetch_desc(&p.seq[i].tk);
       }
       uint32_t it = 0, ul = 0;
-      for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ul) {
+      for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
         const Unit un = decode_unit(p, u);
         const SeqDev& s = p.seq[un.si];
         if (!wait_phase(c, bar(c, B_QFREE), (ul & 1u) ^ 1u, 6)) break;
-        ptx::mbar_expect_tx(bar(c, B_QFULL), kSub * kTileBytes);
+        ptx::mbar_expect_tx(bar(c, B_QFULL), kSub * kQTileBytes);
         for (int b = 0; b < kSub; ++b)
           for (int h2 = 0; h2 < 2; ++h2)
-            ptx::tma_load_3d(sQ + b * kTileBytes + h2 * kHalfBytes, &s.tq, bar(c, B_QFULL), h2 * 64, un.head,
-                             un.qb * kUnitRows + b * kBM);
+            ptx::tma_load_3d(sQ + b * kQTileBytes + h2 * kQHalfBytes, &s.tq, bar(c, B_QFULL), h2 * 64, un.head,
+                             un.qb * kUnitRows + int(rank) * kCtaRows + b * kBM);
         bool ok = true;
         for (int j = 0; j < un.nkt; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_KFREE + st), (n & 1u) ^ 1u, 7)) { ok = false; break; }
-          ptx::mbar_expect_tx(bar(c, B_KFULL + st), kTileBytes);
+          ptx::mbar_expect_tx(bar(c, B_KFULL + st), kKStageBytes);
           for (int h2 = 0; h2 < 2; ++h2)
-            ptx::tma_load_3d(sK + st * kTileBytes + h2 * kHalfBytes, &s.tk, bar(c, B_KFULL + st), h2 * 64, un.head,
-                             j * kBN);
+            ptx::tma_load_3d(sK + st * kKStageBytes + h2 * kKHalfBytes, &s.tk, bar(c, B_KFULL + st), h2 * 64,
+                             un.head, j * kBN + int(rank) * kKRows);
         }
         if (!ok) break;
       }
     } else if (warp == 14 && lane == 0) {
-      // ===================== TMA producer: V =====================
+      // ===================== TMA producer: this CTA's V column half =====================
       for (int i = 0; i < p.n_seqs; ++i) ptx::tma_prefetch_desc(&p.seq[i].tv);
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
         const Unit un = decode_unit(p, u);
         const SeqDev& s = p.seq[un.si];
         for (int j = 0; j < un.nkt; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_VFREE + st), (n & 1u) ^ 1u, 8)) { ok = false; break; }
-          ptx::mbar_expect_tx(bar(c, B_VFULL + st), kTileBytes);
-          for (int h2 = 0; h2 < 2; ++h2)
-            ptx::tma_load_3d(sV + st * kTileBytes + h2 * kHalfBytes, &s.tv, bar(c, B_VFULL + st), h2 * 64, un.head,
-                             j * kBN);
+          ptx::mbar_expect_tx(bar(c, B_VFULL + st), kVStageBytes);
+          ptx::tma_load_3d(sV + st * kVStageBytes, &s.tv, bar(c, B_VFULL + st), int(rank) * 64, un.head, j * kBN);
         }
       }
-    } else if (warp == 13 && lane == 0) {
-      // ===================== MMA issuer =====================
+    } else if (warp == 15 && lane == 0) {
+      // ===================== V landed -> tell the leader =====================
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
+        const Unit un = decode_unit(p, u);
+        for (int j = 0; j < un.nkt; ++j, ++it) {
+          const uint32_t st = it % kStages, n = it / kStages;
+          if (!wait_phase(c, bar(c, B_VFULL + st), n & 1u, 17)) { ok = false; break; }
+          ptx::mbar_arrive_cluster(lbar(B_VREADY + st));
+        }
+      }
+    } else if (warp == 13 && lane == 0 && rank == 0) {
+      // ===================== MMA issuer (leader CTA, for the pair) =====================
       // Waits on smem handoffs (Q/K after RoPE, V after TMA) need no tcgen05
       // fence; waits on TMEM handoffs (P written with tcgen05.st, O read by
       // the epilogue) do.  Descriptors are built once; a k-step only moves
       // the 14-bit start-address field (addresses < 256 KB, so no carry).
-      const uint32_t id_s = ptx::idesc_bf16_f32(kBM, kBN, false);
-      const uint32_t id_pv = ptx::idesc_bf16_f32(kBM, kHD, true);
-      const uint64_t dq0 = desc_kmajor(sQ, 0), dq1 = desc_kmajor(sQ + kTileBytes, 0);
+      const uint32_t id_s = ptx::idesc_bf16_f32(2 * kBM, kBN, false);
+      const uint32_t id_pv = ptx::idesc_bf16_f32(2 * kBM, kHD, true);
+      const uint64_t dq0 = desc_kmajor(sQ), dq1 = desc_kmajor(sQ + kQTileBytes);
+      constexpr uint16_t kBoth = 3;
       uint32_t it = 0, g = 0, ul = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++ul) {
+      for (int u = cluster; ok && u < p.total_units; u += n_clusters, ++ul) {
         const Unit un = decode_unit(p, u);
-        if (!wait_phase(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
+        if (!wait_phase_cluster(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
         for (int j = 0; j < un.nkt; ++j, ++it, ++g) {
           const uint32_t st = it % kStages, n = it / kStages;
-          if (!wait_phase(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
-          const uint64_t dk = desc_kmajor(sK + st * kTileBytes, 0);
+          if (!wait_phase_cluster(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
+          const uint64_t dk = desc_kmajor(sK + st * kKStageBytes);
           if (j > 0) {
             const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
-            if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 11)) { ok = false; break; }
-            const uint64_t dv = desc_v(sV + sp * kTileBytes, 0);
+            if (!wait_phase_cluster(c, bar(c, B_VREADY + sp), np & 1u, 11)) { ok = false; break; }
+            const uint64_t dv = desc_v(sV + sp * kVStageBytes);
             for (int b = 0; b < kSub && ok; ++b) {
-              if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 12)) { ok = false; break; }
+              if (!wait_phase_cluster(c, bar(c, B_PFULL + b), (g - 1) & 1u, 12)) { ok = false; break; }
               if (j == 1) {
-                if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 13)) { ok = false; break; }
+                if (!wait_phase_cluster(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 13)) { ok = false; break; }
               }
               ptx::tc_fence_after();
-              // O_b (+)= P_b(j-1) V(j-1): P from TMEM, V from shared memory (MN-major)
+              // O_b (+)= P_b(j-1) V(j-1): P from each CTA's TMEM, V split by column halves
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)),
-                            id_pv, (j > 1 || kk > 0) ? 1u : 0u);
-              ptx::mma_commit(bar(c, B_ODONE + b));
-              // S_b(j) = Q_b K(j)^T
+                ptx::mma2_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)),
+                             id_pv, (j > 1 || kk > 0) ? 1u : 0u);
+              ptx::mma2_commit_mc(bar(c, B_ODONE + b), kBoth);
+              // S_b(j) = Q_b K(j)^T: Q rows from each CTA, keys split 64 + 64
               const uint64_t dq = b ? dq1 : dq0;
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t off = uint64_t(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
-                ptx::mma_ss(tmem_base + col_s(b), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
-              }
-              ptx::mma_commit(bar(c, B_SFULL + b));
+              for (int kk = 0; kk < 8; ++kk)
+                ptx::mma2_ss(tmem_base + col_s(b), dq + kstep_off(kk, kQHalfBytes), dk + kstep_off(kk, kKHalfBytes),
+                             id_s, kk > 0 ? 1u : 0u);
+              ptx::mma2_commit_mc(bar(c, B_SFULL + b), kBoth);
             }
             if (!ok) break;
-            ptx::mma_commit(bar(c, B_VFREE + sp));
+            ptx::mma2_commit_mc(bar(c, B_VFREE + sp), kBoth);
           } else {
             for (int b = 0; b < kSub; ++b) {
               const uint64_t dq = b ? dq1 : dq0;
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t off = uint64_t(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
-                ptx::mma_ss(tmem_base + col_s(b), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
-              }
-              ptx::mma_commit(bar(c, B_SFULL + b));
+              for (int kk = 0; kk < 8; ++kk)
+                ptx::mma2_ss(tmem_base + col_s(b), dq + kstep_off(kk, kQHalfBytes), dk + kstep_off(kk, kKHalfBytes),
+                             id_s, kk > 0 ? 1u : 0u);
+              ptx::mma2_commit_mc(bar(c, B_SFULL + b), kBoth);
             }
           }
-          ptx::mma_commit(bar(c, B_KFREE + st));
-          if (j == un.nkt - 1) ptx::mma_commit(bar(c, B_QFREE));
+          ptx::mma2_commit_mc(bar(c, B_KFREE + st), kBoth);
+          if (j == un.nkt - 1) ptx::mma2_commit_mc(bar(c, B_QFREE), kBoth);
         }
         if (!ok) break;
         // PV of the unit's last tile
         const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
-        if (!wait_phase(c, bar(c, B_VFULL + sp), np & 1u, 14)) { ok = false; break; }
-        const uint64_t dv = desc_v(sV + sp * kTileBytes, 0);
+        if (!wait_phase_cluster(c, bar(c, B_VREADY + sp), np & 1u, 14)) { ok = false; break; }
+        const uint64_t dv = desc_v(sV + sp * kVStageBytes);
         for (int b = 0; b < kSub && ok; ++b) {
-          if (!wait_phase(c, bar(c, B_PFULL + b), (g - 1) & 1u, 15)) { ok = false; break; }
+          if (!wait_phase_cluster(c, bar(c, B_PFULL + b), (g - 1) & 1u, 15)) { ok = false; break; }
           if (un.nkt == 1) {
-            if (!wait_phase(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 16)) { ok = false; break; }
+            if (!wait_phase_cluster(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 16)) { ok = false; break; }
           }
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            ptx::mma_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)), id_pv,
-                        (un.nkt > 1 || kk > 0) ? 1u : 0u);
-          ptx::mma_commit(bar(c, B_ODONE + b));
+            ptx::mma2_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)), id_pv,
+                         (un.nkt > 1 || kk > 0) ? 1u : 0u);
+          ptx::mma2_commit_mc(bar(c, B_ODONE + b), kBoth);
         }
         if (!ok) break;
-        ptx::mma_commit(bar(c, B_VFREE + sp));
+        ptx::mma2_commit_mc(bar(c, B_VFREE + sp), kBoth);
       }
-      // every tcgen05 op this thread issued is complete before TMEM is freed
-      ptx::mma_commit(bar(c, B_FINAL));
+      // every MMA of the pair is complete before either CTA frees TMEM
+      ptx::mma2_commit_mc(bar(c, B_FINAL), kBoth);
+    }
+    if (warp == 13 && lane == 0) {
       const uint64_t t0 = ptx::globaltimer_ns();
       while (!ptx::mbar_try_wait(bar(c, B_FINAL), 0)) {
-        if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) break;
+        if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
+          *c.abort = 1;
+          atomicCAS(c.p->status, 0, int(RKV_ERR_TIMEOUT) | (18 << 8));
+          break;
+        }
       }
     }
   }
@@ -663,9 +744,11 @@ done:
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_arrive();   // neither CTA leaves while its peer may still use its barriers or TMEM
+  ptx::cluster_wait();
   if (warp == 13) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, kTmemCols);
+    ptx::tmem_dealloc2(tmem_base, kTmemCols);
   }
 }
 
@@ -684,13 +767,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [L][H][128] bf16 view, row stride in elements; box = 128 rows x 1 head x 64 cols.
-static rkv_status make_map(CUtensorMap* m, const void* ptr, int64_t L, int H, int64_t row_stride) {
+// [L][H][128] bf16 view, row stride in elements; box = box_rows rows x 1 head x 64 cols.
+static rkv_status make_map(CUtensorMap* m, const void* ptr, int64_t L, int H, int64_t row_stride, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[3] = {cuuint64_t(kHD), cuuint64_t(H), cuuint64_t(L)};
   cuuint64_t strides[2] = {cuuint64_t(kHD * 2), cuuint64_t(row_stride * 2)};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, cuuint32_t(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -782,14 +865,14 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   for (int oi = 0; oi < n_seqs; ++oi) {
     const rkv_attn_seq& s = seqs[order[oi]];
     SeqDev& d = p.seq[oi];
-    if ((st = make_map(&d.tq, s.q, s.Lq, H, s.q_stride)) != RKV_OK) return st;
-    if ((st = make_map(&d.tk, s.k, s.Lk, H, s.k_stride)) != RKV_OK) return st;
-    if ((st = make_map(&d.tv, s.v, s.Lk, H, s.v_stride)) != RKV_OK) return st;
+    if ((st = make_map(&d.tq, s.q, s.Lq, H, s.q_stride, kBM)) != RKV_OK) return st;
+    if ((st = make_map(&d.tk, s.k, s.Lk, H, s.k_stride, kKRows)) != RKV_OK) return st;
+    if ((st = make_map(&d.tv, s.v, s.Lk, H, s.v_stride, kBN)) != RKV_OK) return st;
     d.o = static_cast<uint8_t*>(s.o);
     d.o_stride_bytes = s.o_stride * 2;
     d.Lq = s.Lq; d.Lk = s.Lk; d.q_t0 = s.q_t0; d.k_t0 = s.k_t0;
     d.q_frame_offset = s.q_frame_offset; d.block_frames = s.block_frames; d.flags = s.flags;
-    d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;
+    d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;   // 512-row blocks, one per CTA pair
     d.unit_begin = int32_t(units);
     units += int64_t(d.n_qblocks) * H;
     if (s.flags & RKV_ROPE_Q) {
@@ -857,8 +940,27 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   auto kern = default_split ? attn_fwd_kernel<22, 21> : attn_fwd_kernel<0, 0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
-  const int grid = int(std::min<int64_t>(units, sm_count()));
-  kern<<<grid, kThreads, kSmemBytes, cs>>>(p);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cluster size)");
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = cs;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // one CTA pair per pair of SMs that can hold it (persistent)
+  int max_clusters = 0;
+  cfg.gridDim = dim3(2 * 74);
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, (void*)kern, &cfg);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+  if (max_clusters < 1) return fail(RKV_ERR_UNSUPPORTED, "no 2-CTA cluster of attn_fwd_kernel fits on this device");
+  cfg.gridDim = dim3(uint32_t(2 * std::min<int64_t>(units, max_clusters)));
+  e = cudaLaunchKernelEx(&cfg, kern, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return RKV_OK;
