@@ -38,6 +38,7 @@ Q_T0, K_T0 = 6, 0
 RING_SLOTS, RING_INSERT = 21, 5
 ATTN_FLOPS = 4.0 * LQ * LK * D * H                 # QK^T and PV, visible pairs only (no mask)
 RING_BYTES = 2 * 2 * RING_INSERT * F * H * D * 2    # (K and V) x (read + write)
+ROPE_BYTES = 2 * (LQ + LK) * H * D * 2               # Q and K rows, read + write
 SEED = 1002
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
@@ -137,7 +138,7 @@ def make_inputs(device):
     return host, devt
 
 
-def cpu_baseline(host, rows=256):
+def cpu_baseline(host, rows=2048):
     """Time the float64 oracle on a bounded sample: RoPE of all 32,760 keys and
     of ``rows`` query rows, then attention for those rows (all 12 heads)."""
     import oracle
@@ -278,6 +279,23 @@ def run_ours(args):
     h2d = sum(v.nbytes for v in host.values())
     d2h = LQ * H * D * 2
 
+    # standalone 3D-RoPE of the step's Q and K (out of place), for its GB/s
+    yq, yk = torch.empty_like(t["q"]), torch.empty_like(t["k"])
+    for _ in range(3):
+        rkv.rope3d_apply(t["q"], yq, t0=Q_T0, rope=rope)
+        rkv.rope3d_apply(t["k"], yk, t0=K_T0, rope=rope)
+    rope_iters = 20
+    rope_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(rope_iters)]
+    torch.cuda.synchronize()
+    for i in range(rope_iters):
+        rope_ev[i][0].record(stream)
+        rkv.rope3d_apply(t["q"], yq, t0=Q_T0, rope=rope)
+        rkv.rope3d_apply(t["k"], yk, t0=K_T0, rope=rope)
+        rope_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rope_ev)
+    del yq, yk
+
     if rank == 0:
         peaks = measured_peaks()
         ms_per_step = total_ms / args.steps
@@ -300,6 +318,9 @@ def run_ours(args):
             "kv_update": {"value": RING_BYTES / (ring_avg * 1e-3) / 1e9, "unit": "GB/s", "avg_us": ring_avg * 1e3,
                           "bytes_per_call": RING_BYTES, "frac_of_measured_hbm": RING_BYTES / (ring_avg * 1e-3) / 1e9 / peaks["hbm"],
                           "frac_of_nominal_8000": RING_BYTES / (ring_avg * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+            "rope3d": {"value": ROPE_BYTES / (rope_ms * 1e-3) / 1e9, "unit": "GB/s", "avg_us": rope_ms * 1e3,
+                       "bytes_per_call": ROPE_BYTES, "what": "rope3d_apply of Q (23,400 rows) + K (32,760 rows)",
+                       "frac_of_measured_hbm": ROPE_BYTES / (rope_ms * 1e-3) / 1e9 / peaks["hbm"]},
             "e2e": {"value": world * ATTN_FLOPS * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": 2 * args.steps,
