@@ -296,6 +296,18 @@ def run_ours(args):
     rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rope_ev)
     del yq, yk
 
+    # ring insert with K rotated on the way in (same bytes as the plain insert)
+    for _ in range(3):
+        rkv.kvcache_ring_update_rope(ring, t["k_new"], t["v_new"], 21, rope, RING_INSERT)
+    rr_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(rope_iters)]
+    torch.cuda.synchronize()
+    for i in range(rope_iters):
+        rr_ev[i][0].record(stream)
+        rkv.kvcache_ring_update_rope(ring, t["k_new"], t["v_new"], 21, rope, RING_INSERT)
+        rr_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ring_rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rr_ev)
+
     if rank == 0:
         peaks = measured_peaks()
         ms_per_step = total_ms / args.steps
@@ -321,6 +333,10 @@ def run_ours(args):
             "rope3d": {"value": ROPE_BYTES / (rope_ms * 1e-3) / 1e9, "unit": "GB/s", "avg_us": rope_ms * 1e3,
                        "bytes_per_call": ROPE_BYTES, "what": "rope3d_apply of Q (23,400 rows) + K (32,760 rows)",
                        "frac_of_measured_hbm": ROPE_BYTES / (rope_ms * 1e-3) / 1e9 / peaks["hbm"]},
+            "kv_update_rope": {"value": RING_BYTES / (ring_rope_ms * 1e-3) / 1e9, "unit": "GB/s",
+                               "avg_us": ring_rope_ms * 1e3, "bytes_per_call": RING_BYTES,
+                               "what": "kvcache_ring_update_rope: 5 raw-K frames rotated into the ring + 5 V frames",
+                               "frac_of_measured_hbm": RING_BYTES / (ring_rope_ms * 1e-3) / 1e9 / peaks["hbm"]},
             "e2e": {"value": world * ATTN_FLOPS * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": 2 * args.steps,
@@ -335,16 +351,24 @@ def run_ours(args):
 
 
 def load_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if the
-    kernel has not changed since it was captured (else null)."""
-    p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
-    if not os.path.exists(p):
-        return None
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the attention source has changed since that capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_fwd_kernel_denoise_23400x32760.md")
+    src = os.path.join(ROOT, "rolling_kv_cache_rope_b200", "csrc", "attn_fwd.cu")
     try:
         with open(p) as f:
-            j = json.load(f)
-        return j.get("dram_bytes_per_launch")
+            kv = dict(line.split(":", 1) for line in f.read().splitlines()
+                      if line.startswith(("source_sha256:", "dram_bytes_per_launch:")))
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
+        return None
+    if kv.get("source_sha256", "").strip() != sha:
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
         return None
 
 

@@ -245,6 +245,34 @@ rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_
                                int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
                                void* stream);
 
+/*
+ * kvcache_ring_update_rope -- kvcache_ring_update with K rotated on the way in.
+ *
+ * Source: the cache holds keys already rotated, so later passes read them
+ * without a RoPE pass, and RoPE and the per-layer cache copy are the two
+ * kernels the pages single out ("Optimizing Real-Time Video Generation on
+ * Trainium Chips", item 6 "Neuron Kernel Interface"; "Amazon and Reactor tune
+ * Trainium for real-time video generation", section "Three problems for
+ * generic compilers").  One pass reads raw K and V once and writes the ring
+ * once: HBM bytes are those of the plain copy.
+ *
+ *   ring, k_new, v_new, new_row_stride, n_frames, n_evicted
+ *                  as for kvcache_ring_update; k_new holds UNROTATED keys
+ *   t0             time index of the first inserted frame: frame i is rotated
+ *                  with t = t0 + i, rows within a frame with their (h, w)
+ *   rope           frame grid and axis split; grid_h*grid_w must equal the
+ *                  ring's tokens_per_frame
+ * The ring's K slots receive exactly what rope3d_apply(k_new) would write
+ * (same arithmetic, same rounding, within 1 bf16 ulp of the exact rotation);
+ * V slots receive v_new unchanged.  Slot, head, count and eviction follow
+ * kvcache_ring_update.
+ * Errors: those of kvcache_ring_update and rope3d_apply, plus
+ * RKV_ERR_INVALID_ARG when the frame grid does not match tokens_per_frame.
+ */
+rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
+                                    int64_t new_row_stride, int32_t n_frames, int32_t t0,
+                                    const rkv_rope3d* rope, int32_t* n_evicted, void* stream);
+
 /* Slot of logical frame j (0 = oldest valid), or -1 when j is not a valid
  * frame or the ring is malformed. */
 int32_t rkv_ring_slot(const rkv_ring* ring, int32_t logical_frame);

@@ -15,6 +15,13 @@ void clear_error();
 rkv_status fail(rkv_status code, const char* fmt, ...);
 rkv_status cuda_fail(cudaError_t e, const char* what);
 
+// ---- host: argument checks and ring bookkeeping shared by several calls ----
+rkv_status check_rope(const rkv_rope3d* rope, int32_t D);          // rope3d.cu
+rkv_status check_ring(const rkv_ring* ring);                       // ring_update.cu
+rkv_status check_ring_insert(const rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
+                             int32_t n_frames);                     // ring_update.cu
+void ring_advance(rkv_ring* ring, int32_t n_frames, int32_t* n_evicted);  // head, count, evicted
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Byte ranges [a, a+na) and [b, b+nb) overlap.

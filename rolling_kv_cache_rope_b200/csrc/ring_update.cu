@@ -70,7 +70,7 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-static rkv_status check_ring(const rkv_ring* r) {
+rkv_status check_ring(const rkv_ring* r) {
   if (!r) return fail(RKV_ERR_INVALID_ARG, "ring is NULL");
   if (!r->k || !r->v) return fail(RKV_ERR_INVALID_ARG, "ring k/v buffer is NULL");
   if (r->slots < 1 || r->tokens_per_frame < 1 || r->H < 1)
@@ -83,6 +83,34 @@ static rkv_status check_ring(const rkv_ring* r) {
   const uint64_t bytes = uint64_t(r->slots) * r->tokens_per_frame * r->H * r->D * 2;
   if (overlaps(r->k, bytes, r->v, bytes)) return fail(RKV_ERR_INVALID_ARG, "ring k and v buffers overlap");
   return RKV_OK;
+}
+
+rkv_status check_ring_insert(const rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
+                             int32_t n_frames) {
+  if (n_frames < 0 || n_frames > ring->slots)
+    return fail(RKV_ERR_INVALID_ARG, "n_frames %d must be in [0, slots=%d]", n_frames, ring->slots);
+  if (n_frames == 0) return RKV_OK;
+  const int64_t row_elems = int64_t(ring->H) * ring->D;
+  if (!k_new || !v_new) return fail(RKV_ERR_INVALID_ARG, "k_new/v_new is NULL");
+  if (!aligned16(k_new) || !aligned16(v_new)) return fail(RKV_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned");
+  if (new_row_stride < row_elems) return fail(RKV_ERR_INVALID_ARG, "new_row_stride < H*D");
+  if ((new_row_stride * 2) % 16 != 0) return fail(RKV_ERR_INVALID_ARG, "rows of k_new/v_new must be 16-byte aligned");
+  const int64_t rows = int64_t(n_frames) * ring->tokens_per_frame;
+  const uint64_t src_bytes = uint64_t((rows - 1) * new_row_stride + row_elems) * 2;
+  const uint64_t ring_bytes = uint64_t(ring->slots) * ring->tokens_per_frame * row_elems * 2;
+  if (overlaps(k_new, src_bytes, ring->k, ring_bytes) || overlaps(k_new, src_bytes, ring->v, ring_bytes) ||
+      overlaps(v_new, src_bytes, ring->k, ring_bytes) || overlaps(v_new, src_bytes, ring->v, ring_bytes))
+    return fail(RKV_ERR_INVALID_ARG, "new frames overlap the ring buffers");
+  if (uint64_t(rows) * (row_elems * 2 / 16) >= (uint64_t(1) << 31))
+    return fail(RKV_ERR_UNSUPPORTED, "insert too large for one launch");
+  return RKV_OK;
+}
+
+void ring_advance(rkv_ring* ring, int32_t n_frames, int32_t* n_evicted) {
+  const int32_t evicted = ring->count + n_frames > ring->slots ? ring->count + n_frames - ring->slots : 0;
+  ring->head = (ring->head + n_frames) % ring->slots;
+  ring->count = ring->count + n_frames < ring->slots ? ring->count + n_frames : ring->slots;
+  if (n_evicted) *n_evicted = evicted;
 }
 
 }  // namespace rkv
@@ -105,23 +133,11 @@ extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, con
   clear_error();
   rkv_status st = check_ring(ring);
   if (st != RKV_OK) return st;
-  if (n_frames < 0 || n_frames > ring->slots)
-    return fail(RKV_ERR_INVALID_ARG, "n_frames %d must be in [0, slots=%d]", n_frames, ring->slots);
-  const int64_t row_elems = int64_t(ring->H) * ring->D;
+  st = check_ring_insert(ring, k_new, v_new, new_row_stride, n_frames);
+  if (st != RKV_OK) return st;
   if (n_frames > 0) {
-    if (!k_new || !v_new) return fail(RKV_ERR_INVALID_ARG, "k_new/v_new is NULL");
-    if (!aligned16(k_new) || !aligned16(v_new)) return fail(RKV_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned");
-    if (new_row_stride < row_elems) return fail(RKV_ERR_INVALID_ARG, "new_row_stride < H*D");
-    if ((new_row_stride * 2) % 16 != 0) return fail(RKV_ERR_INVALID_ARG, "rows of k_new/v_new must be 16-byte aligned");
-    const int64_t rows = int64_t(n_frames) * ring->tokens_per_frame;
-    const uint64_t src_bytes = uint64_t((rows - 1) * new_row_stride + row_elems) * 2;
-    const uint64_t ring_bytes = uint64_t(ring->slots) * ring->tokens_per_frame * row_elems * 2;
-    if (overlaps(k_new, src_bytes, ring->k, ring_bytes) || overlaps(k_new, src_bytes, ring->v, ring_bytes) ||
-        overlaps(v_new, src_bytes, ring->k, ring_bytes) || overlaps(v_new, src_bytes, ring->v, ring_bytes))
-      return fail(RKV_ERR_INVALID_ARG, "new frames overlap the ring buffers");
-    const uint64_t total_vecs = uint64_t(rows) * (row_elems * 2 / 16);
-    if (total_vecs >= (uint64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "insert too large for one launch");
-
+    const int64_t row_elems = int64_t(ring->H) * ring->D;
+    const uint64_t total_vecs = uint64_t(n_frames) * ring->tokens_per_frame * (row_elems * 2 / 16);
     RingCopyArgs a;
     a.src[0] = static_cast<const uint8_t*>(k_new);
     a.src[1] = static_cast<const uint8_t*>(v_new);
@@ -146,9 +162,6 @@ extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, con
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "ring_copy_kernel launch");
   }
-  const int32_t evicted = ring->count + n_frames > ring->slots ? ring->count + n_frames - ring->slots : 0;
-  ring->head = (ring->head + n_frames) % ring->slots;
-  ring->count = ring->count + n_frames < ring->slots ? ring->count + n_frames : ring->slots;
-  if (n_evicted) *n_evicted = evicted;
+  ring_advance(ring, n_frames, n_evicted);
   return RKV_OK;
 }

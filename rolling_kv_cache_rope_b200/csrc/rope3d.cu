@@ -16,14 +16,20 @@
 // bf16 ulp of the exactly rounded value.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace rkv {
 
 struct RopeArgs {
-  const uint8_t* x;
-  uint8_t* y;
+  const uint8_t* x;        // tensor to rotate
+  uint8_t* y;              // its destination (rows, or ring slots in ring mode)
+  const uint8_t* x2;       // ring mode: tensor copied without rotation (V)
+  uint8_t* y2;
   int64_t x_stride_bytes, y_stride_bytes;
+  uint64_t slot_bytes;     // ring mode: bytes of one ring slot (one frame)
+  int32_t ring_head, ring_slots;
   uint32_t L;
   uint32_t cpr;            // 16-byte chunks per row = H * 16
   uint32_t rows_per_cta;
@@ -64,14 +70,62 @@ __device__ __forceinline__ void rotate_pair(float x0, float x1, const TabEntry& 
   if (fabsf(y1) < lim) y1 = dot2_exact(x0, e.s_hi, e.s_lo, x1, e.c_hi, e.c_lo);
 }
 
+// Address of 16-byte chunk `within` of row r (frame f, row in_f of that
+// frame) in the destination: a strided row, or the row's place in ring slot
+// (head + f) mod slots.
+template <bool kRing>
+__device__ __forceinline__ uint8_t* dst_chunk(const RopeArgs& a, uint8_t* base, uint32_t r, uint32_t f, uint32_t in_f,
+                                              uint32_t within) {
+  if (kRing) {
+    int32_t slot = a.ring_head + int32_t(f);
+    if (slot >= a.ring_slots) slot -= a.ring_slots;
+    return base + uint64_t(slot) * a.slot_bytes + (uint64_t(in_f) * a.cpr + within) * 16u;
+  }
+  return base + int64_t(r) * a.y_stride_bytes + uint64_t(within) * 16u;
+}
+
+// Ring mode, second tensor: copy rows [r0, r1) of x2 into the ring unrotated.
+__device__ __forceinline__ void copy_rows_to_ring(const RopeArgs& a, uint32_t r0, uint32_t r1) {
+  const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
+  for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
+    uint4 v[kRopeUnroll];
+    uint8_t* out[kRopeUnroll];
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const uint32_t ci = base + u * kRopeThreads;
+      out[u] = nullptr;
+      if (ci < c_end) {
+        const uint32_t r = fdiv(ci, a.div_cpr);
+        const uint32_t within = ci - r * a.cpr;
+        const uint32_t f = fdiv(r, a.div_F);
+        v[u] = __ldcs(reinterpret_cast<const uint4*>(a.x2 + int64_t(r) * a.x_stride_bytes + uint64_t(within) * 16u));
+        out[u] = dst_chunk<true>(a, a.y2, r, f, r - f * a.F, within);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u)
+      if (out[u]) *reinterpret_cast<uint4*>(out[u]) = v[u];
+  }
+}
+
+// kRing = false: rotate rows of x into rows of y (rope3d_apply).
+// kRing = true: blockIdx.y = 0 rotates x (K) into ring slots of y, blockIdx.y
+// = 1 copies x2 (V) into ring slots of y2 (kvcache_ring_update_rope).
+template <bool kRing>
 __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) {
   extern __shared__ float4 tab_raw[];
   TabEntry* tab = reinterpret_cast<TabEntry*>(tab_raw);
   const uint32_t r0 = blockIdx.x * a.rows_per_cta;
   if (r0 >= a.L) return;
   const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
+  if (kRing && blockIdx.y == 1) {
+    copy_rows_to_ring(a, r0, r1);
+    return;
+  }
 
-  // positions this CTA can reach
+  // positions this CTA can reach: frames f_lo..f_hi; rows h_lo..h_lo+nh-1;
+  // columns w_lo, w_lo+1, ... (mod grid_w), nw of them (w of row r = r mod
+  // grid_w because a frame holds whole grid rows)
   const uint32_t f_lo = fdiv(r0, a.div_F), f_hi = fdiv(r1 - 1, a.div_F);
   const int32_t nt = int32_t(f_hi - f_lo) + 1;
   int32_t h_lo = 0, nh = a.grid_h;
@@ -79,9 +133,14 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) 
     h_lo = int32_t(fdiv(r0 - f_lo * a.F, a.div_W));
     nh = int32_t(fdiv(r1 - 1 - f_lo * a.F, a.div_W)) - h_lo + 1;
   }
+  int32_t w_lo = 0, nw = a.grid_w;
+  if (r1 - r0 < uint32_t(a.grid_w)) {
+    w_lo = int32_t(r0 - fdiv(r0, a.div_W) * uint32_t(a.grid_w));
+    nw = int32_t(r1 - r0);
+  }
   const int32_t base_h = nt * a.pt;
   const int32_t base_w = base_h + nh * a.ph;
-  const int32_t n_entries = base_w + a.grid_w * a.pw;
+  const int32_t n_entries = base_w + nw * a.pw;
 
   for (int32_t e = threadIdx.x; e < n_entries; e += kRopeThreads) {
     int32_t pos, i, n;
@@ -93,7 +152,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) 
       i = (e - base_h) - hh * a.ph; n = a.ph; pos = h_lo + hh;
     } else {
       const int32_t ww = (e - base_w) / a.pw;
-      i = (e - base_w) - ww * a.pw; n = a.pw; pos = ww;
+      i = (e - base_w) - ww * a.pw; n = a.pw;
+      pos = w_lo + ww;
+      if (pos >= a.grid_w) pos -= a.grid_w;
     }
     const double ang = double(pos) * exp2(-(double(i) / double(n)) * a.log2_theta);
     double s, c;
@@ -129,9 +190,11 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) 
       const uint32_t in_f = r - f * a.F;
       const uint32_t hh = fdiv(in_f, a.div_W);
       const uint32_t ww = in_f - hh * uint32_t(a.grid_w);
+      int32_t wi_off = int32_t(ww) - w_lo;
+      if (wi_off < 0) wi_off += a.grid_w;
       const int32_t ti = int32_t(f - f_lo) * a.pt;
       const int32_t hi = base_h + (int32_t(hh) - h_lo) * a.ph - a.pt;
-      const int32_t wi = base_w + int32_t(ww) * a.pw - a.pt - a.ph;
+      const int32_t wi = base_w + wi_off * a.pw - a.pt - a.ph;
       const int32_t p0 = int32_t(within[u] & 15u) * 4;   // first rotary pair of this chunk
       uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
@@ -143,7 +206,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) 
         rotate_pair(bf16lo_to_f32(w4[k]), bf16hi_to_f32(w4[k]), e, y0, y1);
         w4[k] = pack_bf16x2(y0, y1);
       }
-      *reinterpret_cast<uint4*>(a.y + int64_t(r) * a.y_stride_bytes + uint64_t(within[u]) * 16u) =
+      *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, within[u])) =
           make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
   }
@@ -165,6 +228,50 @@ rkv_status check_rope(const rkv_rope3d* rope, int32_t D) {
   if (rope->pairs_t + rope->pairs_h + rope->pairs_w != D / 2)
     return fail(RKV_ERR_INVALID_ARG, "pairs_t+pairs_h+pairs_w must equal D/2");
   if (!(rope->theta > 1.0f) || !isfinite(rope->theta)) return fail(RKV_ERR_INVALID_ARG, "theta must be finite and > 1");
+  return RKV_OK;
+}
+
+// Fill the rotation part of RopeArgs, pick rows per CTA under the table
+// budget and launch (ring mode: two CTA rows, K rotated and V copied).
+template <bool kRing>
+static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
+                              cudaStream_t stream) {
+  a.L = uint32_t(L);
+  a.cpr = uint32_t(H) * 16u;
+  a.F = uint32_t(rope->grid_h) * uint32_t(rope->grid_w);
+  a.t0 = t0;
+  a.grid_h = rope->grid_h;
+  a.grid_w = rope->grid_w;
+  a.pt = rope->pairs_t;
+  a.ph = rope->pairs_h;
+  a.pw = rope->pairs_w;
+  a.log2_theta = log2(double(rope->theta));
+  a.div_F = make_fastdiv(a.F);
+  a.div_W = make_fastdiv(uint32_t(rope->grid_w));
+  a.div_cpr = make_fastdiv(a.cpr);
+  const int64_t target_ctas = int64_t(sm_count()) * 4;
+  int64_t rpc = (L + target_ctas - 1) / target_ctas;
+  if (rpc < 1) rpc = 1;
+  // upper bound of the table a CTA of `rows` rows builds (see the kernel)
+  auto entries = [&](int64_t rows) {
+    const int64_t nt = rows / a.F + 2;
+    return nt * a.pt + int64_t(a.grid_h) * a.ph + std::min<int64_t>(a.grid_w, rows) * a.pw;
+  };
+  if (entries(1) > kRopeMaxEntries) return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
+  while (rpc > 1 && entries(rpc) > kRopeMaxEntries) rpc = (rpc + 1) / 2;
+  a.rows_per_cta = uint32_t(rpc);
+  const int64_t grid = (L + rpc - 1) / rpc;
+  const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kRopeMaxEntries * int(sizeof(TabEntry)));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
+    attr_set = true;
+  }
+  rope3d_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), kRopeThreads, smem, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
   return RKV_OK;
 }
 
@@ -194,47 +301,43 @@ extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H,
   const int64_t last_t = int64_t(t0) + (L - 1) / (int64_t(rope->grid_h) * rope->grid_w);
   if (last_t > INT32_MAX) return fail(RKV_ERR_INVALID_ARG, "time index overflows int32");
 
-  RopeArgs a;
+  RopeArgs a{};
   a.x = static_cast<const uint8_t*>(x);
   a.y = static_cast<uint8_t*>(y);
   a.x_stride_bytes = x_row_stride * 2;
   a.y_stride_bytes = y_row_stride * 2;
-  a.L = uint32_t(L);
-  a.cpr = uint32_t(H) * 16u;
-  a.F = uint32_t(rope->grid_h) * uint32_t(rope->grid_w);
-  a.t0 = t0;
-  a.grid_h = rope->grid_h;
-  a.grid_w = rope->grid_w;
-  a.pt = rope->pairs_t;
-  a.ph = rope->pairs_h;
-  a.pw = rope->pairs_w;
-  a.log2_theta = log2(double(rope->theta));
-  a.div_F = make_fastdiv(a.F);
-  a.div_W = make_fastdiv(uint32_t(rope->grid_w));
-  a.div_cpr = make_fastdiv(a.cpr);
-  const int64_t target_ctas = int64_t(sm_count()) * 4;
-  int64_t rpc = (L + target_ctas - 1) / target_ctas;
-  if (rpc < 1) rpc = 1;
-  // keep the per-CTA table within budget: shrink the row block if needed
-  auto entries = [&](int64_t rows) {
-    const int64_t nt = rows / a.F + 2;
-    return nt * a.pt + int64_t(a.grid_h) * a.ph + int64_t(a.grid_w) * a.pw;
-  };
-  if (int64_t(a.grid_w) * a.pw + 2 * a.pt + int64_t(a.grid_h) * a.ph > kRopeMaxEntries)
-    return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
-  while (rpc > 1 && entries(rpc) > kRopeMaxEntries) rpc = (rpc + 1) / 2;
-  a.rows_per_cta = uint32_t(rpc);
-  const int64_t grid = (L + rpc - 1) / rpc;
-  const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kRopeMaxEntries * int(sizeof(TabEntry)));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
-    attr_set = true;
+  return launch_rope<false>(a, L, H, t0, rope, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
+                                               int64_t new_row_stride, int32_t n_frames, int32_t t0,
+                                               const rkv_rope3d* rope, int32_t* n_evicted, void* stream) {
+  clear_error();
+  rkv_status st = check_ring(ring);
+  if (st != RKV_OK) return st;
+  st = check_rope(rope, ring->D);
+  if (st != RKV_OK) return st;
+  if (int64_t(rope->grid_h) * rope->grid_w != ring->tokens_per_frame)
+    return fail(RKV_ERR_INVALID_ARG, "grid_h*grid_w (%d*%d) must equal tokens_per_frame (%d)", rope->grid_h,
+                rope->grid_w, ring->tokens_per_frame);
+  st = check_ring_insert(ring, k_new, v_new, new_row_stride, n_frames);
+  if (st != RKV_OK) return st;
+  if (n_frames > 0) {
+    if (int64_t(t0) + n_frames - 1 > INT32_MAX) return fail(RKV_ERR_INVALID_ARG, "time index overflows int32");
+    RopeArgs a{};
+    a.x = static_cast<const uint8_t*>(k_new);
+    a.y = static_cast<uint8_t*>(ring->k);
+    a.x2 = static_cast<const uint8_t*>(v_new);
+    a.y2 = static_cast<uint8_t*>(ring->v);
+    a.x_stride_bytes = new_row_stride * 2;
+    a.y_stride_bytes = int64_t(ring->H) * ring->D * 2;
+    a.slot_bytes = uint64_t(ring->tokens_per_frame) * ring->H * ring->D * 2;
+    a.ring_head = ring->head;
+    a.ring_slots = ring->slots;
+    st = launch_rope<true>(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope,
+                           static_cast<cudaStream_t>(stream));
+    if (st != RKV_OK) return st;
   }
-  rope3d_kernel<<<uint32_t(grid), kRopeThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
+  ring_advance(ring, n_frames, n_evicted);
   return RKV_OK;
 }

@@ -61,6 +61,9 @@ _lib.rkv_attn_status.argtypes = [_c.c_void_p, _c.c_void_p]
 _lib.kvcache_ring_update.restype = _c.c_int
 _lib.kvcache_ring_update.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
                                      _c.POINTER(_c.c_int32), _c.c_void_p]
+_lib.kvcache_ring_update_rope.restype = _c.c_int
+_lib.kvcache_ring_update_rope.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
+                                          _c.c_int32, _c.POINTER(rkv_rope3d), _c.POINTER(_c.c_int32), _c.c_void_p]
 _lib.rkv_ring_slot.restype = _c.c_int32
 _lib.rkv_ring_slot.argtypes = [_c.POINTER(rkv_ring), _c.c_int32]
 _lib.rkv_last_error_string.restype = _c.c_char_p
@@ -207,9 +210,7 @@ class KVRing:
         return self.c.count * self.c.tokens_per_frame
 
 
-def kvcache_ring_update(ring, k_new, v_new, n_frames=None, stream=None):
-    """Insert n_frames frames ([n*F, H, D] bf16 CUDA tensors) into ``ring``;
-    returns the number of frames evicted."""
+def _ring_insert_args(ring, k_new, v_new, n_frames):
     ks, vs = _rows(k_new, "k_new"), _rows(v_new, "v_new")
     if ks != vs:
         raise ValueError("k_new and v_new must share a row stride")
@@ -218,7 +219,25 @@ def kvcache_ring_update(ring, k_new, v_new, n_frames=None, stream=None):
         n_frames = k_new.shape[0] // F
     if k_new.shape[0] < n_frames * F or v_new.shape[0] < n_frames * F:
         raise ValueError("k_new/v_new hold fewer than n_frames frames")
+    return ks, int(n_frames)
+
+
+def kvcache_ring_update(ring, k_new, v_new, n_frames=None, stream=None):
+    """Insert n_frames frames ([n*F, H, D] bf16 CUDA tensors) into ``ring``;
+    returns the number of frames evicted."""
+    ks, n_frames = _ring_insert_args(ring, k_new, v_new, n_frames)
     ev = ctypes.c_int32(0)
-    _check(_lib.kvcache_ring_update(ctypes.byref(ring.c), k_new.data_ptr(), v_new.data_ptr(), ks, int(n_frames),
+    _check(_lib.kvcache_ring_update(ctypes.byref(ring.c), k_new.data_ptr(), v_new.data_ptr(), ks, n_frames,
                                     ctypes.byref(ev), _stream(stream)))
+    return ev.value
+
+
+def kvcache_ring_update_rope(ring, k_new, v_new, t0, rope, n_frames=None, stream=None):
+    """Insert n_frames frames like kvcache_ring_update, rotating the raw keys
+    k_new by RoPE3D on the way in (frame i at time t0 + i); returns the
+    number of frames evicted."""
+    ks, n_frames = _ring_insert_args(ring, k_new, v_new, n_frames)
+    ev = ctypes.c_int32(0)
+    _check(_lib.kvcache_ring_update_rope(ctypes.byref(ring.c), k_new.data_ptr(), v_new.data_ptr(), ks, n_frames,
+                                         int(t0), ctypes.byref(rope), ctypes.byref(ev), _stream(stream)))
     return ev.value

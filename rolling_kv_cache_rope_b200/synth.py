@@ -18,13 +18,16 @@ from dataclasses import dataclass
 import numpy as np
 
 
-def bf16_normal_bits(seed, shape):
-    """uint16 bf16 patterns of N(0,1) float32 draws (PCG64(seed)), RNE-rounded."""
-    rng = np.random.Generator(np.random.PCG64(int(seed)))
+def _normal_bits(rng, shape):
     f = rng.standard_normal(size=shape, dtype=np.float32)
     u = f.view(np.uint32)
     r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
+
+
+def bf16_normal_bits(seed, shape):
+    """uint16 bf16 patterns of N(0,1) float32 draws (PCG64(seed)), RNE-rounded."""
+    return _normal_bits(np.random.Generator(np.random.PCG64(int(seed))), shape)
 
 
 @dataclass(frozen=True)
@@ -109,6 +112,19 @@ class Sweep:
     def k_frames_after(self, step):
         """Valid ring frames once ``step`` has inserted its frames."""
         return min(self.ring_slots, self.seed_frames + self.insert * (step + 1))
+
+    def step_inputs(self, layer, step):
+        """bf16 bits of (q, k_new, v_new) of (layer, step): [rows, heads, head_dim]
+        arrays drawn in that order from one PCG64(seed(layer, step)) stream.
+        Step -1 is the pre-seeded frame(s): q is None and k/v hold seed_frames
+        frames; other steps draw q_frames query frames and insert frames."""
+        rng = np.random.Generator(np.random.PCG64(self.seed(layer, step)))
+        F, H, D = self.frame_tokens, self.heads, self.head_dim
+        n = self.seed_frames if step < 0 else self.insert
+        q = None if step < 0 else _normal_bits(rng, (self.q_frames * F, H, D))
+        k = _normal_bits(rng, (n * F, H, D))
+        v = _normal_bits(rng, (n * F, H, D))
+        return q, k, v
 
 
 SWEEP = Sweep()

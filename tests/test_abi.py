@@ -131,6 +131,37 @@ def test_rope_zero_rows_is_a_noop(rkv):
     assert rkv.lib().rope3d_apply(None, None, 0, 2, 128, 256, 256, 0, ctypes.byref(r), None) == rkv.RKV_OK
 
 
+@pytest.mark.parametrize("change,n,t0,rope_kw,frag", [
+    ({}, 6, 0, {}, "n_frames"),
+    ({}, 2, 0, {"grid_h": 5}, "tokens_per_frame"),
+    ({}, 2, 0, {"pairs": (22, 21, 20)}, "pairs"),
+    ({"D": 64}, 2, 0, {}, "head_dim"),
+    ({"head": 9}, 2, 0, {}, "head"),
+    ({}, 2, 2**31 - 1, {}, "overflows"),
+])
+def test_ring_update_rope_rejects(rkv, change, n, t0, rope_kw, frag):
+    lib = rkv.lib()
+    r = ring(rkv, **change)
+    rp = rope(rkv, **rope_kw)
+    before = (r.head, r.count)
+    ev = ctypes.c_int32(-7)
+    st = lib.kvcache_ring_update_rope(ctypes.byref(r), fake(0x40000000), fake(0x50000000), 2 * 128, n, t0,
+                                      ctypes.byref(rp), ctypes.byref(ev), None)
+    assert st == rkv.RKV_ERR_INVALID_ARG, rkv.rkv_last_error_string()
+    assert frag in rkv.rkv_last_error_string()
+    assert (r.head, r.count) == before and ev.value == -7
+
+
+def test_ring_update_rope_zero_frames_is_a_host_noop(rkv):
+    lib = rkv.lib()
+    r = ring(rkv, head=2, count=4)
+    rp = rope(rkv)
+    ev = ctypes.c_int32(-1)
+    assert lib.kvcache_ring_update_rope(ctypes.byref(r), None, None, 256, 0, 0, ctypes.byref(rp), ctypes.byref(ev),
+                                        None) == rkv.RKV_OK
+    assert (r.head, r.count, ev.value) == (2, 4, 0)
+
+
 def seq(rkv, **kw):
     base = dict(q=0x100000, k=0x200000, v=0x300000, o=0x400000, q_stride=256, k_stride=256, v_stride=256,
                 o_stride=256, Lq=72, Lk=120, q_t0=2, k_t0=0, q_frame_offset=2, block_frames=0, flags=3,
