@@ -158,16 +158,14 @@ __device__ __forceinline__ uint32_t bar(const Ctx& c, int i) { return c.bar0 + 8
 __device__ __forceinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t parity, int where) {
   if (ptx::mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
-  uint32_t spins = 0;
   while (true) {
-    if (ptx::mbar_try_wait(b, parity)) return true;
-    if ((++spins & 15u) == 0) {
-      if (*c.abort) return false;
-      if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
-        *c.abort = 1;
-        atomicCAS(c.p->status, 0, int(RKV_ERR_TIMEOUT) | (where << 8));
-        return false;
-      }
+    // sleeps in hardware until the phase completes (at most ~20 us per try)
+    if (ptx::mbar_try_wait_sleep(b, parity, 20000u)) return true;
+    if (*c.abort) return false;
+    if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
+      *c.abort = 1;
+      atomicCAS(c.p->status, 0, int(RKV_ERR_TIMEOUT) | (where << 8));
+      return false;
     }
   }
 }
