@@ -308,6 +308,15 @@ def run_ours(args):
     torch.cuda.synchronize()
     ring_rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rr_ev)
 
+    # kernels per step: attention, the merge of split tail units when the
+    # persistent grid's last wave is at most half full (same rule as the
+    # library, one CTA pair per two SMs), and the ring update
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    clusters, units = sms // 2, -(-LQ // 512) * H
+    rest = units % clusters
+    split = units > clusters and rest > 0 and 2 * rest <= clusters and ws.numel() > 256
+    launches_per_step = 3 if split else 2
+
     if rank == 0:
         peaks = measured_peaks()
         ms_per_step = total_ms / args.steps
@@ -339,7 +348,7 @@ def run_ours(args):
                                "frac_of_measured_hbm": RING_BYTES / (ring_rope_ms * 1e-3) / 1e9 / peaks["hbm"]},
             "e2e": {"value": world * ATTN_FLOPS * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -149,10 +149,14 @@ typedef struct {
  *   H >= 1, D == 128, softmax_scale > 0 (1/sqrt(128) for SDPA)
  *   rope           frame grid / axis split; required (also defines F for the
  *                  mask) even when no sequence sets a RoPE flag
- *   workspace      device memory of at least attn_fwd_varlen_workspace_size()
- *                  bytes, 16-byte aligned, not used by another call in flight;
- *                  holds the device status word.  May be NULL only when that
- *                  size is 0.
+ *   workspace      device memory, 16-byte aligned, not used by another call
+ *                  in flight; at least 256 bytes (the device status word).
+ *                  attn_fwd_varlen_workspace_size() bytes (about 20 MB on a
+ *                  B200) also hold partial results for the tail of the
+ *                  persistent grid: when the last wave of work units is at
+ *                  most half full, those units run as two halves over their
+ *                  key tiles and a second kernel merges the halves.  With a
+ *                  smaller workspace the call runs without that split.
  * A query row that sees no key gets zeros.  Precision: bf16 operands, fp32
  * accumulation and softmax, bf16 output.
  * Errors: RKV_ERR_INVALID_ARG (shapes, pointers, alignment, overlap of o with
@@ -194,8 +198,11 @@ rkv_status rkv_attn_status(void* workspace, void* stream);
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents.  Calls that overlap on the GPU (on different streams, or
  * from different host threads without ordering) race on it; serialise them.
- * Limit: a launch whose scratch need (attn_fwd_varlen_workspace_size) exceeds
- * 256 bytes is rejected with RKV_ERR_UNSUPPORTED.
+ * Limit: the array holds only the 256 bytes a launch needs at least, so these
+ * launches never split the tail of the grid (see attn_fwd_varlen's workspace)
+ * and can be a few percent slower on full-size work; a launch whose minimum
+ * scratch need exceeded the array would be rejected with
+ * RKV_ERR_UNSUPPORTED.
  * A device-side timeout stops the kernel as in attn_fwd_varlen but is only
  * recorded in the internal array; callers that need it reported back use
  * attn_fwd_varlen with their own workspace and rkv_attn_status.

@@ -110,7 +110,13 @@ struct SeqDev {
 
 struct Params {
   SeqDev seq[RKV_MAX_SEQS];
-  int32_t n_seqs, H, total_units;
+  int32_t n_seqs, H;
+  // work items: units [0, n_whole) whole, then each of the remaining
+  // n_split units as two items over the first and second half of its key
+  // tiles, whose partial results go to part_o / part_ml
+  int32_t total_units, n_whole, n_split;
+  float* part_o;     // [2 * n_split][kUnitRows][kHD] unnormalised O
+  float* part_ml;    // [2 * n_split][kUnitRows][2] running max (log2 units) and row sum
   float scale_log2;
   int32_t grid_h, grid_w;
   int32_t t_lo, n_t;
@@ -185,6 +191,8 @@ __device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t b, uint32_t par
 
 struct Unit {
   int si, head, qb, nkt;
+  int kt0, kt1;   // key tiles [kt0, kt1) of this work item
+  int part;       // -1: whole unit; else index of the item's partial-result slot
 };
 
 __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p, int row) {
@@ -199,8 +207,14 @@ __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p
 // sequence (all query blocks of head 0, then head 1, ...), so the clusters in
 // flight at any time share the K/V tiles of one or two heads in L2.  Masked
 // sequences list their query blocks from the most to the least visible keys.
-__device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
+__device__ __forceinline__ Unit decode_unit(const Params& p, int item) {
   Unit r;
+  int u = item;
+  r.part = -1;
+  if (item >= p.n_whole) {   // half of a split unit
+    r.part = item - p.n_whole;
+    u = p.n_whole + (r.part >> 1);
+  }
   int si = 0;
   while (si + 1 < p.n_seqs && u >= p.seq[si + 1].unit_begin) ++si;
   const SeqDev& s = p.seq[si];
@@ -213,6 +227,12 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   if (last > s.Lq - 1) last = s.Lq - 1;
   const int64_t kv = row_kv_limit(s, p, last);
   r.nkt = int((kv + kBN - 1) / kBN);
+  r.kt0 = 0;
+  r.kt1 = r.nkt;
+  if (r.part >= 0) {
+    if (r.part & 1) r.kt0 = r.nkt / 2;
+    else r.kt1 = r.nkt / 2;
+  }
   return r;
 }
 
@@ -342,6 +362,34 @@ __device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uin
   return (a01.x + a01.y) + (a23.x + a23.y);
 }
 
+// exp_store_tile<false> that also returns the row max of the raw scores in
+// mx: the exponentials use the running max m_use and are kept unless the
+// tile's own max exceeds it by more than the rescale threshold.
+__device__ __forceinline__ float exp_store_tile_max(const uint32_t (&sr)[4][32], uint32_t tS, float scale_log2,
+                                                    float m_use, float& mx) {
+  const float2 sc2 = make_float2(scale_log2, scale_log2);
+  const float2 nm2 = make_float2(-m_use, -m_use);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float s0 = __uint_as_float(sr[ch][2 * i]), s1 = __uint_as_float(sr[ch][2 * i + 1]);
+      mx4[i & 3] = max3f(mx4[i & 3], s0, s1);
+      const float2 x = __ffma2_rn(make_float2(s0, s1), sc2, nm2);
+      const float2 pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));
+      acc[i & 3] = __fadd2_rn(acc[i & 3], pp);
+      pk[i] = pack_bf16x2(pp.x, pp.y);
+    }
+    ptx::tmem_st16(tS + ch * 16, pk);   // P (bf16) overwrites S columns 0..63
+  }
+  mx = fmaxf(max3f(mx4[0], mx4[1], mx4[2]), mx4[3]);
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  return (a01.x + a01.y) + (a23.x + a23.y);
+}
+
 // K-major operand (rows of 128 bf16 in two 64-column 128B-swizzled halves):
 // 8-row groups 1024 bytes apart; k-step kk starts 32 bytes further inside a
 // half, or in the second half from kk = 4.
@@ -459,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int qrow = un.qb * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
       const int64_t my_limit = row_kv_limit(s, p, qrow < s.Lq ? qrow : s.Lq - 1);
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < un.nkt; ++j, ++g) {
+      for (int j = un.kt0; j < un.kt1; ++j, ++g) {
         if (!wait_warp(c, bar(c, B_SFULL + wg), g & 1u, 1)) goto done;
         ptx::tc_fence_after();
         uint32_t sr[4][32];
@@ -469,28 +517,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int64_t kbase = int64_t(j) * kBN;
         const int lim = kbase + kBN > my_limit ? int(my_limit - kbase) : kBN;
         const bool masked = __any_sync(0xffffffffu, lim < kBN);
-        if (masked) {
+        const float m_old = m;
+        float m_new, tile_sum;
+        bool need;
+        if (j > un.kt0 && !masked) {
+          // speculative: exponentials against the running max while the
+          // tile max is found; redone (rarely) when the max has to move
+          float mx;
+          tile_sum = exp_store_tile_max(sr, tS, scale_log2, m, mx);
+          m_new = fmaxf(m, mx * scale_log2);
+          need = m_new > m + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            if (need) m = m_new;
+            tile_sum = exp_store_tile<false>(sr, tS, scale_log2, m);
+          }
+        } else {
+          if (masked) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
+          }
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
+            for (int i = 0; i < 32; i += 2)
+              mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], __uint_as_float(sr[ch][i]), __uint_as_float(sr[ch][i + 1]));
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          m_new = fmaxf(m, mx * scale_log2);
+          need = m_new > m + kRescaleLog2;
+          if (need) m = m_new;
+          const float m_use = (m == -INFINITY) ? 0.f : m;
+          tile_sum = masked ? exp_store_tile<false>(sr, tS, scale_log2, m_use)
+                            : exp_store_tile<kPolyExp>(sr, tS, scale_log2, m_use);
         }
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], __uint_as_float(sr[ch][i]), __uint_as_float(sr[ch][i + 1]));
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const float m_new = fmaxf(m, mx * scale_log2);
-        const bool need = m_new > m + kRescaleLog2;
-        const float m_old = m;
-        if (need) m = m_new;
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        const float tile_sum = masked ? exp_store_tile<false>(sr, tS, scale_log2, m_use)
-                                      : exp_store_tile<kPolyExp>(sr, tS, scale_log2, m_use);
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (j > un.kt0 && __any_sync(0xffffffffu, need)) {
           // O holds tiles 0..j-1 scaled to the old max: wait for the last PV,
           // then rescale in TMEM (PV(j) is not issued before P_FULL below)
           if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 2)) goto done;
@@ -526,7 +589,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(ofree);   // O may now be overwritten
-        if (qrow < s.Lq) {
+        if (un.part >= 0) {
+          // half of a split unit: unnormalised O, running max and row sum
+          // for the combine pass
+          const int64_t prow = int64_t(un.part) * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
+          uint4* dst = reinterpret_cast<uint4*>(p.part_o + prow * kHD);
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[ch * 8 + i] = make_uint4(r[ch][4 * i], r[ch][4 * i + 1], r[ch][4 * i + 2], r[ch][4 * i + 3]);
+          reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(m, l);
+        } else if (qrow < s.Lq) {
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t pk[16];
@@ -567,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       ptx::fence_proxy_async_smem();
       ptx::named_sync(1, 128);
       if (rt == 0) ptx::mbar_arrive_cluster(qready);
-      for (int j = 0; j < un.nkt; ++j, ++it) {
+      for (int j = un.kt0; j < un.kt1; ++j, ++it) {
         const uint32_t st = it % kStages, n = it / kStages;
         if (!wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5)) goto done;
         if (s.flags & RKV_ROPE_K) {
@@ -609,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             ptx::tma_load_3d(sQ + b * kQTileBytes + h2 * kQHalfBytes, &s.tq, bar(c, B_QFULL), h2 * 64, un.head,
                              un.qb * kUnitRows + int(rank) * kCtaRows + b * kBM);
         bool ok = true;
-        for (int j = 0; j < un.nkt; ++j, ++it) {
+        for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_KFREE + st), (n & 1u) ^ 1u, 7)) { ok = false; break; }
           ptx::mbar_expect_tx(bar(c, B_KFULL + st), kKStageBytes);
@@ -627,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
         const Unit un = decode_unit(p, u);
         const SeqDev& s = p.seq[un.si];
-        for (int j = 0; j < un.nkt; ++j, ++it) {
+        for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_VFREE + st), (n & 1u) ^ 1u, 8)) { ok = false; break; }
           ptx::mbar_expect_tx(bar(c, B_VFULL + st), kVStageBytes);
@@ -640,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       bool ok = true;
       for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
         const Unit un = decode_unit(p, u);
-        for (int j = 0; j < un.nkt; ++j, ++it) {
+        for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_VFULL + st), n & 1u, 17)) { ok = false; break; }
           ptx::mbar_arrive_cluster(lbar(B_VREADY + st));
@@ -661,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int u = cluster; ok && u < p.total_units; u += n_clusters, ++ul) {
         const Unit un = decode_unit(p, u);
         if (!wait_phase_cluster(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
-        for (int j = 0; j < un.nkt; ++j, ++it, ++g) {
+        const int nk = un.kt1 - un.kt0;   // tiles of this item; j counts them from 0
+        for (int j = 0; j < nk; ++j, ++it, ++g) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase_cluster(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
           const uint64_t dk = desc_kmajor(sK + st * kKStageBytes);
@@ -702,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
           }
           ptx::mma2_commit_mc(bar(c, B_KFREE + st), kBoth);
-          if (j == un.nkt - 1) ptx::mma2_commit_mc(bar(c, B_QFREE), kBoth);
+          if (j == nk - 1) ptx::mma2_commit_mc(bar(c, B_QFREE), kBoth);
         }
         if (!ok) break;
         // PV of the unit's last tile
@@ -711,14 +786,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const uint64_t dv = desc_v(sV + sp * kVStageBytes);
         for (int b = 0; b < kSub && ok; ++b) {
           if (!wait_phase_cluster(c, bar(c, B_PFULL + b), (g - 1) & 1u, 15)) { ok = false; break; }
-          if (un.nkt == 1) {
+          if (nk == 1) {
             if (!wait_phase_cluster(c, bar(c, B_OFREE + b), (ul & 1u) ^ 1u, 16)) { ok = false; break; }
           }
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             ptx::mma2_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)), id_pv,
-                         (un.nkt > 1 || kk > 0) ? 1u : 0u);
+                         (nk > 1 || kk > 0) ? 1u : 0u);
           ptx::mma2_commit_mc(bar(c, B_ODONE + b), kBoth);
         }
         if (!ok) break;
@@ -787,6 +862,90 @@ static int sm_count() {
 }
 
 constexpr size_t kWorkspaceBytes = 256;
+constexpr int kMaxSplit = 64;   // split units per launch at most
+constexpr size_t kPartBytesPerItem = size_t(kUnitRows) * (kHD * 4 + 8);
+
+// Combine the two halves of each split unit: per query row, with M the larger
+// running max, O = (O_a 2^(m_a - M) + O_b 2^(m_b - M)) / (l_a 2^(m_a - M) +
+// l_b 2^(m_b - M)) -> bf16 -> the output row (the same merge the online
+// softmax applies between key tiles).
+struct CombineUnit {
+  uint8_t* o;
+  int64_t o_stride_bytes;
+  int32_t Lq, head, row0, pad;
+};
+struct CombineArgs {
+  const float* part_o;
+  const float2* part_ml;
+  int32_t n_split;
+  CombineUnit unit[kMaxSplit];
+};
+
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __grid_constant__ CombineArgs a) {
+  const int64_t idx = int64_t(blockIdx.x) * kCombineThreads + threadIdx.x;   // (unit, row, 8-column group)
+  if (idx >= int64_t(a.n_split) * kUnitRows * (kHD / 8)) return;
+  const int u = int(idx / (kUnitRows * (kHD / 8)));
+  const int rem = int(idx - int64_t(u) * kUnitRows * (kHD / 8));
+  const int row = rem / (kHD / 8), cg = rem % (kHD / 8);
+  const CombineUnit& cu = a.unit[u];
+  const int qrow = cu.row0 + row;
+  if (qrow >= cu.Lq) return;
+  const int64_t ra = int64_t(2 * u) * kUnitRows + row, rb = ra + kUnitRows;
+  const float2 mla = a.part_ml[ra], mlb = a.part_ml[rb];
+  const float mx = fmaxf(mla.x, mlb.x);
+  const float wa = mla.y > 0.f ? exp2f(mla.x - mx) : 0.f;
+  const float wb = mlb.y > 0.f ? exp2f(mlb.x - mx) : 0.f;
+  const float lsum = mla.y * wa + mlb.y * wb;
+  const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+  const float4* oa = reinterpret_cast<const float4*>(a.part_o + ra * kHD + cg * 8);
+  const float4* ob = reinterpret_cast<const float4*>(a.part_o + rb * kHD + cg * 8);
+  const float4 a0 = oa[0], a1 = oa[1], b0 = ob[0], b1 = ob[1];
+  const float ca = wa * inv, cb = wb * inv;
+  uint4 out;
+  out.x = pack_bf16x2(a0.x * ca + b0.x * cb, a0.y * ca + b0.y * cb);
+  out.y = pack_bf16x2(a0.z * ca + b0.z * cb, a0.w * ca + b0.w * cb);
+  out.z = pack_bf16x2(a1.x * ca + b1.x * cb, a1.y * ca + b1.y * cb);
+  out.w = pack_bf16x2(a1.z * ca + b1.z * cb, a1.w * ca + b1.w * cb);
+  *reinterpret_cast<uint4*>(cu.o + int64_t(qrow) * cu.o_stride_bytes + int64_t(cu.head) * (kHD * 2) + cg * 16) = out;
+}
+
+// Launch shape of the attention kernel (attributes set, cluster of 2) and the
+// number of clusters that fit on the current device at once.
+static rkv_status attn_launch_shape(bool default_split, cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr,
+                                    const void*& kern_ptr, int& max_clusters) {
+  auto kern = default_split ? attn_fwd_kernel<22, 21> : attn_fwd_kernel<0, 0>;
+  kern_ptr = reinterpret_cast<const void*>(kern);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cluster size)");
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(2 * 74);
+  max_clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, kern_ptr, &cfg);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+  if (max_clusters < 1) return fail(RKV_ERR_UNSUPPORTED, "no 2-CTA cluster of attn_fwd_kernel fits on this device");
+  return RKV_OK;
+}
+
+// Units of the last, partly filled wave of the persistent grid that are run as
+// two half-units (split over their key tiles) so the wave finishes in about
+// half the time; 0 when the last wave is more than half full.
+static int tail_split_units(int64_t units, int clusters) {
+  if (clusters < 2 || units <= clusters) return 0;
+  const int64_t rest = units % clusters;
+  if (rest == 0 || 2 * rest > clusters) return 0;
+  return int(std::min<int64_t>(rest, kMaxSplit));
+}
 
 }  // namespace attn
 }  // namespace rkv
@@ -795,7 +954,18 @@ using namespace rkv;
 using namespace rkv::attn;
 
 extern "C" size_t attn_fwd_varlen_workspace_size(const rkv_attn_seq*, int32_t, int32_t, int32_t) {
-  return kWorkspaceBytes;
+  // the status word, plus room for the partial results of the largest tail
+  // split this device can take (half of its concurrent CTA pairs)
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  const void* kern = nullptr;
+  int clusters = 0;
+  if (attn_launch_shape(true, cfg, attr, kern, clusters) != RKV_OK) {
+    clear_error();
+    return kWorkspaceBytes;
+  }
+  const int split = std::min(clusters / 2, kMaxSplit);
+  return kWorkspaceBytes + size_t(2 * split) * kPartBytesPerItem;
 }
 
 static rkv_status validate_seq(const rkv_attn_seq& s, int i, int32_t H) {
@@ -918,7 +1088,6 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   }
   p.n_seqs = n_seqs;
   p.H = H;
-  p.total_units = int32_t(units);
   p.scale_log2 = float(double(softmax_scale) * 1.4426950408889634);
   p.grid_h = rope->grid_h; p.grid_w = rope->grid_w;
   p.t_lo = int32_t(t_lo); p.n_t = int32_t(n_t);
@@ -931,36 +1100,68 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   p.timeout_ns = 2000000000ull;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kWorkspaceBytes, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
   // the 22/21/21 split of the pages' 128-dim heads gets its own instantiation
   const bool default_split = rope->pairs_t == 22 && rope->pairs_h == 21 && rope->pairs_w == 21;
-  auto kern = default_split ? attn_fwd_kernel<22, 21> : attn_fwd_kernel<0, 0>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cluster size)");
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = cs;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // one CTA pair per pair of SMs that can hold it (persistent)
+  const void* kern = nullptr;
   int max_clusters = 0;
-  cfg.gridDim = dim3(2 * 74);
-  e = cudaOccupancyMaxActiveClusters(&max_clusters, (void*)kern, &cfg);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-  if (max_clusters < 1) return fail(RKV_ERR_UNSUPPORTED, "no 2-CTA cluster of attn_fwd_kernel fits on this device");
-  cfg.gridDim = dim3(uint32_t(2 * std::min<int64_t>(units, max_clusters)));
-  e = cudaLaunchKernelEx(&cfg, kern, p);
-  e = cudaGetLastError();
+  if ((st = attn_launch_shape(default_split, cfg, attr, kern, max_clusters)) != RKV_OK) return st;
+  cfg.stream = cs;
+
+  // tail split: the last n_split units run as two half-units each when the
+  // workspace can hold their partial results and every such unit has >= 2
+  // key tiles
+  int n_split = tail_split_units(units, max_clusters);
+  if (workspace_bytes < kWorkspaceBytes + size_t(2 * n_split) * kPartBytesPerItem) n_split = 0;
+  CombineArgs ca;
+  memset(&ca, 0, sizeof(ca));
+  for (int k = 0; k < n_split; ++k) {
+    const int64_t u = units - n_split + k;
+    int si = 0;
+    while (si + 1 < n_seqs && u >= p.seq[si + 1].unit_begin) ++si;
+    const SeqDev& d = p.seq[si];
+    const int64_t local = u - d.unit_begin;
+    const int head = int(local / d.n_qblocks);
+    const int ord = int(local - int64_t(head) * d.n_qblocks);
+    const int qb = d.block_frames > 0 ? (d.n_qblocks - 1 - ord) : ord;
+    int64_t last = int64_t(qb + 1) * kUnitRows - 1;
+    if (last > d.Lq - 1) last = d.Lq - 1;
+    int64_t kv = d.Lk;
+    if (d.block_frames > 0) {
+      const int64_t qf = int64_t(d.q_frame_offset) + last / F;
+      kv = std::min<int64_t>((qf / d.block_frames + 1) * d.block_frames * F, d.Lk);
+    }
+    if ((kv + kBN - 1) / kBN < 2) { n_split = 0; break; }
+    ca.unit[k].o = d.o;
+    ca.unit[k].o_stride_bytes = d.o_stride_bytes;
+    ca.unit[k].Lq = d.Lq;
+    ca.unit[k].head = head;
+    ca.unit[k].row0 = qb * kUnitRows;
+  }
+  ca.n_split = n_split;
+  p.n_whole = int32_t(units - n_split);
+  p.n_split = n_split;
+  p.total_units = int32_t(units + n_split);
+  p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceBytes);
+  p.part_ml = p.part_o + size_t(2 * n_split) * kUnitRows * kHD;
+  ca.part_o = p.part_o;
+  ca.part_ml = reinterpret_cast<const float2*>(p.part_ml);
+
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kWorkspaceBytes, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  // one CTA pair per pair of SMs that can hold it (persistent)
+  cfg.gridDim = dim3(uint32_t(2 * std::min<int64_t>(p.total_units, max_clusters)));
+  e = default_split ? cudaLaunchKernelEx(&cfg, attn_fwd_kernel<22, 21>, p)
+                    : cudaLaunchKernelEx(&cfg, attn_fwd_kernel<0, 0>, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  if (n_split > 0) {
+    const int64_t threads = int64_t(n_split) * kUnitRows * (kHD / 8);
+    attn_combine_kernel<<<uint32_t((threads + kCombineThreads - 1) / kCombineThreads), kCombineThreads, 0, cs>>>(ca);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "attn_combine_kernel launch");
+  }
   return RKV_OK;
 }
 
@@ -1023,7 +1224,9 @@ static rkv_status noalloc_scratch(void** out) {
 extern "C" rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
                                               float softmax_scale, const rkv_rope3d* rope, void* stream) {
   clear_error();
-  const size_t need = attn_fwd_varlen_workspace_size(seqs, n_seqs, H, D);
+  // the launch needs kWorkspaceBytes at least; with no room for partial
+  // results it runs without the tail split
+  const size_t need = kWorkspaceBytes;
   if (need > kNoAllocScratchBytes)
     return fail(RKV_ERR_UNSUPPORTED, "this launch needs %zu bytes of scratch; the no-alloc entry point has %zu",
                 need, kNoAllocScratchBytes);
