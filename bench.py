@@ -334,6 +334,40 @@ def run_ours(args):
     torch.cuda.synchronize()
     ring_rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rr_ev)
 
+    def time_attn(seqs_, iters=5):
+        for _ in range(3):
+            rkv.attn_fwd_varlen(seqs_, rope, workspace=ws)
+        evs_ = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+        torch.cuda.synchronize()
+        for i in range(iters):
+            evs_[i][0].record(stream)
+            rkv.attn_fwd_varlen(seqs_, rope, workspace=ws)
+            evs_[i][1].record(stream)
+        torch.cuda.synchronize()
+        rkv.rkv_attn_status(ws)
+        return statistics.mean(e[0].elapsed_time(e[1]) for e in evs_)
+
+    # the rolling-cache pass: keys already rotated (as the rotated ring insert
+    # stores them), only Q rotated in-kernel, same sizes as the step
+    seq_qonly = rkv.AttnSeq(t["q"], t["k"], t["v"], o, q_t0=Q_T0, k_t0=K_T0, rope_k=False)
+    qonly_ms = time_attn([seq_qonly])
+    # the batched two-pass launch: the denoise pass and a 5-frame cache-update
+    # pass over the same 21-frame context, both frame-block-causal (blocks of
+    # 3 frames, query frames bottom-right aligned); FLOPs of visible pairs only
+    gen = torch.Generator(device=device).manual_seed(SEED + 1)
+    q_cache = torch.randn((5 * F, H, D), generator=gen, device=device).to(torch.bfloat16)
+    o_cache = torch.empty_like(q_cache)
+    two_pass = [rkv.AttnSeq(t["q"], t["k"], t["v"], o, q_t0=Q_T0, k_t0=K_T0, block_frames=3,
+                            q_frame_offset=LK // F - LQ // F),
+                 rkv.AttnSeq(q_cache, t["k"], t["v"], o_cache, q_t0=16, k_t0=K_T0, block_frames=3,
+                             q_frame_offset=16)]
+
+    def visible_pairs(q_frames, off, k_frames, block=3):
+        return sum(F * F for qf in range(q_frames) for kf in range(k_frames) if kf // block <= (off + qf) // block)
+
+    two_pass_flops = 4.0 * D * H * (visible_pairs(LQ // F, LK // F - LQ // F, LK // F) + visible_pairs(5, 16, LK // F))
+    two_pass_ms = time_attn(two_pass)
+
     # kernels per step: attention, the merge of split tail units when the
     # persistent grid's last wave is at most half full (same rule as the
     # library, one CTA pair per two SMs), and the ring update
@@ -368,6 +402,14 @@ def run_ours(args):
             "rope3d": {"value": ROPE_BYTES / (rope_ms * 1e-3) / 1e9, "unit": "GB/s", "avg_us": rope_ms * 1e3,
                        "bytes_per_call": ROPE_BYTES, "what": "rope3d_apply of Q (23,400 rows) + K (32,760 rows)",
                        "frac_of_measured_hbm": ROPE_BYTES / (rope_ms * 1e-3) / 1e9 / peaks["hbm"]},
+            "attn_k_prerotated": {"value": ATTN_FLOPS / (qonly_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                  "avg_ms": qonly_ms, "what": "same attention with K already rotated "
+                                                              "(rolling-cache pass: Q-only RoPE in-kernel)",
+                                  "frac_of_nominal_2250": ATTN_FLOPS / (qonly_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS},
+            "two_pass": {"value": two_pass_flops / (two_pass_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                         "avg_ms": two_pass_ms, "useful_flops": two_pass_flops,
+                         "what": "one launch: denoise 23,400 + cache-update 7,800 queries over 32,760 keys, "
+                                 "frame-block-causal (3 frames), RoPE on Q and K; visible pairs only"},
             "kv_update_rope": {"value": RING_BYTES / (ring_rope_ms * 1e-3) / 1e9, "unit": "GB/s",
                                "avg_us": ring_rope_ms * 1e3, "bytes_per_call": RING_BYTES,
                                "what": "kvcache_ring_update_rope: 5 raw-K frames rotated into the ring + 5 V frames",
