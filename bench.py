@@ -186,6 +186,18 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(ms, world, device):
+    """The largest of the ranks' device-timed milliseconds (every rank calls
+    this at the same point; world == 1 returns ms unchanged)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -242,10 +254,7 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     ring_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, device)
 
     # end to end through the public API with host buffers: every step copies
     # its inputs (Q, K, V, new K/V frames) from pinned host memory, runs the
@@ -297,10 +306,8 @@ def run_ours(args):
     e2e_run(e2e_steps, e0, e1)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
     if world > 1:
-        tt = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
     h2d = sum(v.nbytes for v in host.values())
     d2h = LQ * H * D * 2
