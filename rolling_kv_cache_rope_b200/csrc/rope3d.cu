@@ -41,7 +41,11 @@ struct RopeArgs {
   FastDiv div_F, div_W, div_cpr;
 };
 
-constexpr int kRopeThreads = 256;
+// threads per CTA: the standalone op runs one 1024-thread CTA per SM (each
+// cos/sin table serves more rows); the ring insert, a short launch with a V
+// copy beside it, keeps four 256-thread CTAs per SM (measured faster there)
+template <bool kRing>
+constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
 constexpr int kRopeMaxEntries = 4096;  // 64 KB of float4 per CTA
 
@@ -86,6 +90,7 @@ __device__ __forceinline__ uint8_t* dst_chunk(const RopeArgs& a, uint8_t* base, 
 
 // Ring mode, second tensor: copy rows [r0, r1) of x2 into the ring unrotated.
 __device__ __forceinline__ void copy_rows_to_ring(const RopeArgs& a, uint32_t r0, uint32_t r1) {
+  constexpr int kRopeThreads = rope_threads<true>();
   const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
   for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
     uint4 v[kRopeUnroll];
@@ -112,7 +117,8 @@ __device__ __forceinline__ void copy_rows_to_ring(const RopeArgs& a, uint32_t r0
 // kRing = true: blockIdx.y = 0 rotates x (K) into ring slots of y, blockIdx.y
 // = 1 copies x2 (V) into ring slots of y2 (kvcache_ring_update_rope).
 template <bool kRing>
-__global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const RopeArgs a) {
+__global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const RopeArgs a) {
+  constexpr int kRopeThreads = rope_threads<kRing>();
   extern __shared__ float4 tab_raw[];
   TabEntry* tab = reinterpret_cast<TabEntry*>(tab_raw);
   const uint32_t r0 = blockIdx.x * a.rows_per_cta;
@@ -249,7 +255,7 @@ static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, con
   a.div_F = make_fastdiv(a.F);
   a.div_W = make_fastdiv(uint32_t(rope->grid_w));
   a.div_cpr = make_fastdiv(a.cpr);
-  const int64_t target_ctas = int64_t(sm_count()) * 4;
+  const int64_t target_ctas = int64_t(sm_count()) * (kRing ? 4 : 1);
   int64_t rpc = (L + target_ctas - 1) / target_ctas;
   if (rpc < 1) rpc = 1;
   // upper bound of the table a CTA of `rows` rows builds (see the kernel)
@@ -269,7 +275,7 @@ static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, con
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
     attr_set = true;
   }
-  rope3d_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), kRopeThreads, smem, stream>>>(a);
+  rope3d_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
   return RKV_OK;
