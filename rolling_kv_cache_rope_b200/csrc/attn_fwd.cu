@@ -36,10 +36,17 @@
 // of the same S region, and the PV MMA takes P straight from TMEM.  While one
 // softmax warpgroup works, the tensor cores run the other sub-tile's MMAs
 // (ping-pong).  The running max is only moved (and O rescaled in TMEM) when it
-// grows by more than 2^8.  Operand readiness is reported to the leader with
+// grows by more than 2^8; after a unit's first tile the exponentials are taken
+// against the running max while the tile max is found, and redone in the rare
+// case it has to move.  Operand readiness is reported to the leader with
 // cluster-scope mbarrier arrives; the leader's commits are multicast to both
-// CTAs.  No TMA load uses multicast.  All waits are bounded: a stuck wait makes
-// the CTA stop, records RKV_ERR_TIMEOUT in the workspace and frees TMEM.
+// CTAs.  No TMA load uses multicast.  Waiting threads sleep in mbarrier
+// try_wait (suspend-time hint).  All waits are bounded: a stuck wait makes the
+// CTA stop, records RKV_ERR_TIMEOUT in the workspace and frees TMEM.
+// Tail of the persistent grid: when its last wave of units is at most half
+// full, those units run as two halves over their key tiles, leave
+// unnormalised O, running max and row sum in the workspace, and
+// attn_combine_kernel merges each pair into the output.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
