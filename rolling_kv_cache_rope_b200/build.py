@@ -5,7 +5,7 @@
 The library links the CUDA runtime statically and reaches the driver's
 cuTensorMapEncodeTiled through cudaGetDriverEntryPoint, so it loads on a
 machine without a GPU (calls then fail with RKV_ERR_CUDA) and needs no
-LD_LIBRARY_PATH on the GPU machine.
+LD_LIBRARY_PATH where a GPU is present.
 """
 
 import argparse
