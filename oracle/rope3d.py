@@ -21,6 +21,12 @@ design notes):
   one-axis RoPE frequency law applied to an axis of 2n dimensions);
 * rotation is y0 = x0 cos a - x1 sin a, y1 = x0 sin a + x1 cos a; V is not
   rotated.
+
+Two variants the pages leave open are also computed here (the layout and the
+frequency base are the two free choices of the reading above): the
+"rotate-half" pair layout, where pair j holds elements (j, j + D/2) instead
+of (2j, 2j+1), and a frequency base per axis, theta = (theta_t, theta_h,
+theta_w).
 """
 
 import numpy as np
@@ -48,20 +54,25 @@ def pair_axes(pairs):
 
 
 def rope_angles(token_index, t0, grid_h, grid_w, pairs, theta):
-    """Rotation angle of every (token, pair): float64 [len(token_index), sum(pairs)]."""
+    """Rotation angle of every (token, pair): float64 [len(token_index), sum(pairs)].
+
+    ``theta`` is one frequency base for all axes or a (t, h, w) triple."""
     t, h, w = token_positions(token_index, t0, grid_h, grid_w)
     pos = np.stack([t, h, w], axis=1).astype(np.float64)            # [L, 3]
     axis, local, count = pair_axes(pairs)
-    freq = np.power(np.float64(theta), -local.astype(np.float64) / count.astype(np.float64))
+    bases = np.broadcast_to(np.asarray(theta, dtype=np.float64), (3,))
+    freq = np.power(bases[axis], -local.astype(np.float64) / count.astype(np.float64))
     return pos[:, axis] * freq[None, :]                               # [L, P]
 
 
-def rope3d_ref(x, t0, grid_h, grid_w, pairs=(22, 21, 21), theta=10000.0, token_index=None):
+def rope3d_ref(x, t0, grid_h, grid_w, pairs=(22, 21, 21), theta=10000.0, token_index=None, layout="adjacent"):
     """Rotate x (float64 [L, H, D]) by the 3D-RoPE of its tokens.
 
     ``token_index`` gives each row's index within its sequence (default
-    0..L-1); it lets a caller rotate a sample of rows.  Returns float64, same
-    shape.  D must equal 2 * sum(pairs).
+    0..L-1); it lets a caller rotate a sample of rows.  ``theta``: one base or
+    a (t, h, w) triple.  ``layout``: "adjacent" (pair j = elements 2j, 2j+1)
+    or "half" (pair j = elements j, j + D/2).  Returns float64, same shape.
+    D must equal 2 * sum(pairs).
     """
     x = np.asarray(x, dtype=np.float64)
     L, H, D = x.shape
@@ -72,9 +83,15 @@ def rope3d_ref(x, t0, grid_h, grid_w, pairs=(22, 21, 21), theta=10000.0, token_i
     ang = rope_angles(token_index, t0, grid_h, grid_w, pairs, theta)  # [L, P]
     c = np.cos(ang)[:, None, :]
     s = np.sin(ang)[:, None, :]
-    x0 = x[..., 0::2]
-    x1 = x[..., 1::2]
+    if layout == "adjacent":
+        first, second = slice(0, D, 2), slice(1, D, 2)
+    elif layout == "half":
+        first, second = slice(0, D // 2), slice(D // 2, D)
+    else:
+        raise ValueError("layout must be 'adjacent' or 'half'")
+    x0 = x[..., first]
+    x1 = x[..., second]
     y = np.empty_like(x)
-    y[..., 0::2] = x0 * c - x1 * s
-    y[..., 1::2] = x0 * s + x1 * c
+    y[..., first] = x0 * c - x1 * s
+    y[..., second] = x0 * s + x1 * c
     return y

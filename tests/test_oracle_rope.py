@@ -133,3 +133,68 @@ def test_rows_subset_equals_full():
     full = rope3d_ref(x, 2, 4, 6, PAIRS)
     part = rope3d_ref(x[rows], 2, 4, 6, PAIRS, token_index=rows)
     assert np.array_equal(full[rows], part)
+
+
+# ---- rotate-half layout and per-axis frequency bases -------------------------
+
+def test_rotate_half_is_adjacent_after_interleaving():
+    # moving element j to 2j and element j + D/2 to 2j + 1 turns the
+    # rotate-half layout into the adjacent one, for any input and position
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((50, 3, D))
+    perm = np.empty(D, dtype=np.int64)
+    perm[0::2] = np.arange(D // 2)
+    perm[1::2] = np.arange(D // 2) + D // 2
+    half = rope3d_ref(x, 4, 5, 6, PAIRS, layout="half")
+    adj = rope3d_ref(x[..., perm], 4, 5, 6, PAIRS, layout="adjacent")
+    back = np.empty_like(adj)
+    back[..., perm] = adj
+    np.testing.assert_allclose(half, back, rtol=0, atol=1e-15)
+
+
+def test_rotate_half_unit_vector_textbook_values():
+    # (1, 0) in pair 30 (an h pair: local index 8 of 21), i.e. element 30 in
+    # the rotate-half layout; on a 10x1 grid token 7 is row 7: the pair turns
+    # by 7 * 10000^(-8/21) and lands on elements 30 and 30 + 64 only
+    x = np.zeros((8, 1, D))
+    x[:, 0, 30] = 1.0
+    y = rope3d_ref(x, 0, 10, 1, PAIRS, layout="half")
+    a = 7 * 10000.0 ** (-8 / 21)
+    assert abs(y[7, 0, 30] - math.cos(a)) < 1e-15 and abs(y[7, 0, 30 + 64] - math.sin(a)) < 1e-15
+    assert np.count_nonzero(np.abs(y[7, 0]) > 1e-15) == 2
+
+
+def test_per_axis_theta_closed_form_and_default():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((40, 2, D))
+    same = rope3d_ref(x, 2, 4, 6, PAIRS, theta=(10000.0, 10000.0, 10000.0))
+    np.testing.assert_array_equal(same, rope3d_ref(x, 2, 4, 6, PAIRS, theta=10000.0))
+    # h pair with local index 7 of 21 (global pair 29) under theta_h = 100:
+    # frequency 100^(-1/3) = 0.2154...; token 13 on a 4x6 grid is row 2
+    u = np.zeros((14, 1, D))
+    u[:, 0, 2 * 29] = 1.0
+    y = rope3d_ref(u, 0, 4, 6, PAIRS, theta=(10000.0, 100.0, 10000.0))
+    ang = math.atan2(y[13, 0, 2 * 29 + 1], y[13, 0, 2 * 29])
+    assert abs(ang - 2 * 100.0 ** (-1 / 3)) < 1e-12
+    # the t and w pairs do not see theta_h
+    z = rope3d_ref(x, 2, 4, 6, PAIRS, theta=(10000.0, 100.0, 10000.0))
+    ref = rope3d_ref(x, 2, 4, 6, PAIRS, theta=10000.0)
+    t_and_w = np.r_[0:44, 86:128]
+    np.testing.assert_array_equal(z[..., t_and_w], ref[..., t_and_w])
+
+
+@pytest.mark.parametrize("layout,theta", [("half", 10000.0), ("adjacent", (500.0, 2000.0, 30000.0)),
+                                          ("half", (500.0, 2000.0, 30000.0))])
+def test_variants_keep_norms_and_relative_positions(layout, theta):
+    rng = np.random.default_rng(13)
+    F = 24
+    q = rng.standard_normal((1, 1, D))
+    k = rng.standard_normal((1, 1, D))
+    nq = np.linalg.norm(rope3d_ref(np.repeat(q, 60, 0), 0, 4, 6, PAIRS, theta, layout=layout), axis=-1)
+    np.testing.assert_allclose(nq, np.linalg.norm(q), rtol=1e-12)
+    # score between token a and token b depends only on their (t, h, w) offset
+    def score(ta, tb):
+        xq = rope3d_ref(q, 0, 4, 6, PAIRS, theta, token_index=np.array([ta]), layout=layout)
+        xk = rope3d_ref(k, 0, 4, 6, PAIRS, theta, token_index=np.array([tb]), layout=layout)
+        return float(np.sum(xq * xk))
+    assert abs(score(7, 7 + F + 7) - score(2 * F + 7, 3 * F + 14)) < 1e-9
