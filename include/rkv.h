@@ -61,14 +61,24 @@ typedef enum {
  *   pairs use t, the next pairs_h use h, the last pairs_w use w
  *   (pairs_t + pairs_h + pairs_w == D/2; 22/21/21 for D = 128);
  *   pair with local index k on an axis with n pairs turns by
- *       angle = pos * theta^(-k/n)
+ *       angle = pos * theta_axis^(-k/n)   (theta_axis = theta unless the
+ *       per-axis bases below are set)
  *   y0 = x0 cos(angle) - x1 sin(angle);  y1 = x0 sin(angle) + x1 cos(angle).
  */
 typedef struct {
   int32_t grid_h, grid_w;            /* frame grid; tokens per frame = grid_h*grid_w */
   int32_t pairs_t, pairs_h, pairs_w; /* rotary pairs per axis, sum = D/2            */
-  float theta;                       /* frequency base, 10000 for all three axes    */
+  float theta;                       /* frequency base of the t axis (and of h, w
+                                        when theta_h / theta_w are 0); 10000        */
+  float theta_h, theta_w;            /* frequency bases of the h and w axes; 0 =
+                                        theta                                       */
+  int32_t layout;                    /* RKV_ROPE_ADJACENT or RKV_ROPE_HALF          */
 } rkv_rope3d;
+
+/* rkv_rope3d.layout: which elements form rotary pair j (0 <= j < D/2) */
+#define RKV_ROPE_ADJACENT 0 /* elements 2j and 2j+1 (the reading above)            */
+#define RKV_ROPE_HALF 1     /* elements j and j + D/2 ("rotate-half"); the pages
+                               leave the layout open, so both are offered      */
 
 /*
  * rope3d_apply -- y = RoPE3D(x) for every row and head.

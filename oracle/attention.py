@@ -65,7 +65,7 @@ def attention_ref(q, k, v, scale, visible=None, row_chunk=512):
 
 def fused_attention_ref(q_raw, k_raw, v, *, scale, grid_h, grid_w,
                         rope_q, rope_k, q_t0, k_t0, pairs=(22, 21, 21), theta=10000.0,
-                        block_frames=0, q_frame_offset=0, rows=None):
+                        block_frames=0, q_frame_offset=0, rows=None, layout="adjacent"):
     """One sequence of the batched launch: optional RoPE on Q/K, mask, attention.
 
     Inputs are float64 [L, H, D] (the exact values of the bf16 inputs).  The
@@ -81,10 +81,10 @@ def fused_attention_ref(q_raw, k_raw, v, *, scale, grid_h, grid_w,
     rows = np.asarray(rows, dtype=np.int64)
     qs = q_raw[rows]
     if rope_q:
-        qs = rope3d_ref(qs, q_t0, grid_h, grid_w, pairs, theta, token_index=rows)
+        qs = rope3d_ref(qs, q_t0, grid_h, grid_w, pairs, theta, token_index=rows, layout=layout)
     ks = k_raw
     if rope_k:
-        ks = rope3d_ref(k_raw, k_t0, grid_h, grid_w, pairs, theta)
+        ks = rope3d_ref(k_raw, k_t0, grid_h, grid_w, pairs, theta, layout=layout)
     visible = None
     if block_frames > 0:
         visible = frame_block_visible(Lq, Lk, grid_h * grid_w, q_frame_offset,

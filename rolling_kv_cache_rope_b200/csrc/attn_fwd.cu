@@ -140,7 +140,7 @@ struct Params {
   int8_t ch_ax_lo[16], ch_ax_hi[16], ch_sel[16];
   uint32_t F;
   FastDiv div_F, div_W;
-  double log2_theta;
+  double log2_theta[3];   // frequency base per axis (t, h, w)
   int32_t* status;
   uint64_t timeout_ns;
 };
@@ -321,6 +321,84 @@ __device__ __forceinline__ void rope_row(const Params& p, uint32_t tabC, uint32_
   }
 }
 
+// Rotate 4 rotary pairs of the rotate-half layout: element e (0..3) of the
+// 8-byte word pair a (first 64 columns) with element e of b (columns + 64).
+__device__ __forceinline__ void rotate_half4(uint32_t& a0, uint32_t& a1, uint32_t& b0, uint32_t& b1, float4 C,
+                                             float4 S) {
+  const uint32_t aw[2] = {a0, a1}, bw[2] = {b0, b1};
+  uint32_t ao[2], bo[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float2 x0 = make_float2(bf16lo_to_f32(aw[h]), bf16hi_to_f32(aw[h]));
+    const float2 x1 = make_float2(bf16lo_to_f32(bw[h]), bf16hi_to_f32(bw[h]));
+    const float2 nx1 = make_float2(-x1.x, -x1.y);
+    const float2 c = h ? make_float2(C.z, C.w) : make_float2(C.x, C.y);
+    const float2 s = h ? make_float2(S.z, S.w) : make_float2(S.x, S.y);
+    const float2 y0 = __ffma2_rn(x0, c, __fmul2_rn(nx1, s));   // x0 cos - x1 sin
+    const float2 y1 = __ffma2_rn(x0, s, __fmul2_rn(x1, c));    // x0 sin + x1 cos
+    ao[h] = pack_bf16x2(y0.x, y0.y);
+    bo[h] = pack_bf16x2(y1.x, y1.y);
+  }
+  a0 = ao[0]; a1 = ao[1]; b0 = bo[0]; b1 = bo[1];
+}
+
+// cos / sin of table chunk tc (rotary pairs 4tc..4tc+3) for a row at (pt, ph, pw).
+template <int kPT, int kPH>
+__device__ __forceinline__ void tab_chunk(const Params& p, uint32_t tabC, uint32_t tabS, int tc, int pt, int ph, int pw,
+                                          float4& C, float4& S) {
+  int alo, ahi;
+  if (kPT > 0) {
+    alo = (4 * tc) < kPT ? 0 : ((4 * tc) < kPT + kPH ? 1 : 2);
+    ahi = (4 * tc + 3) < kPT ? 0 : ((4 * tc + 3) < kPT + kPH ? 1 : 2);
+  } else {
+    alo = p.ch_ax_lo[tc];
+    ahi = p.ch_ax_hi[tc];
+  }
+  const uint32_t e_lo = uint32_t(p.ch_base_lo[tc] + pick3(alo, pt, ph, pw)) * 16u;
+  C = ptx::lds128f(tabC + e_lo);
+  S = ptx::lds128f(tabS + e_lo);
+  if (alo != ahi) {
+    const uint32_t e_hi = uint32_t(p.ch_base_hi[tc] + pick3(ahi, pt, ph, pw)) * 16u;
+    const float4 C2 = ptx::lds128f(tabC + e_hi);
+    const float4 S2 = ptx::lds128f(tabS + e_hi);
+    C = make_float4(C.x * C2.x, C.y * C2.y, C.z * C2.z, C.w * C2.w);
+    S = make_float4(S.x + S2.x, S.y + S2.y, S.z + S2.z, S.w + S2.w);
+  }
+}
+
+// rope_row for the rotate-half layout: chunk pairs g in [kG0, kG0 + kGN)
+// (g < 8): chunk g of the first 64 columns holds elements 8g..8g+7, chunk g of
+// the second half the elements 64 later; pair 8g + e rotates the two
+// elements e.  Table chunks 2g and 2g + 1 give the cos / sin of the 8 pairs.
+template <int kPT, int kPH, int kG0, int kGN>
+__device__ __forceinline__ void rope_row_half(const Params& p, uint32_t tabC, uint32_t tabS, uint32_t row_addr,
+                                              uint32_t half_stride, uint32_t swz, int pt, int ph, int pw) {
+#pragma unroll
+  for (int g0 = kG0; g0 < kG0 + kGN; g0 += 2) {
+    uint4 va[2], vb[2];
+    uint32_t aa[2], ab[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int g = g0 + x;
+      aa[x] = row_addr + ((uint32_t(g) ^ swz) << 4);
+      ab[x] = aa[x] + half_stride;
+      va[x] = ptx::lds128(aa[x]);
+      vb[x] = ptx::lds128(ab[x]);
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int g = g0 + x;
+      float4 C0, S0, C1, S1;
+      tab_chunk<kPT, kPH>(p, tabC, tabS, 2 * g, pt, ph, pw, C0, S0);
+      tab_chunk<kPT, kPH>(p, tabC, tabS, 2 * g + 1, pt, ph, pw, C1, S1);
+      rotate_half4(va[x].x, va[x].y, vb[x].x, vb[x].y, C0, S0);
+      rotate_half4(va[x].z, va[x].w, vb[x].z, vb[x].w, C1, S1);
+      ptx::sts128(aa[x], va[x]);
+      ptx::sts128(ab[x], vb[x]);
+    }
+  }
+}
+
 // (t, h, w) table positions of token `row` of a sequence whose first frame is t0.
 __device__ __forceinline__ void row_positions(const Params& p, int row, int t0, int& pt, int& ph, int& pw) {
   const uint32_t f = fdiv(uint32_t(row), p.div_F);
@@ -419,7 +497,7 @@ __device__ __forceinline__ void setmaxnreg_dec_producer() {
 }
 
 // kPT/kPH: compile-time RoPE axis split (pairs on t and h), or 0/0 for any split
-template <int kPT, int kPH>
+template <int kPT, int kPH, bool kHalf>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -481,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int i = 4 * chunk + j - p.ax_first[a];
       double sd = 0.0, cd = 1.0;
       if (i >= 0 && i < p.ax_count[a])
-        sincos(double(pos) * exp2(-(double(i) / double(p.ax_count[a])) * p.log2_theta), &sd, &cd);
+        sincos(double(pos) * exp2(-(double(i) / double(p.ax_count[a])) * p.log2_theta[a]), &sd, &cd);
       cs[j] = __double2float_rn(cd);
       sn[j] = __double2float_rn(sd);
     }
@@ -640,8 +718,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           if (row < s.Lq) {
             int pt, ph, pw;
             row_positions(p, row, s.q_t0, pt, ph, pw);
-            rope_row<kPT, kPH, 0, 16>(p, sTabC, sTabS, sQ + uint32_t(b * kQTileBytes + rt * 128), kQHalfBytes,
-                                      uint32_t(rt & 7), pt, ph, pw);
+            if (kHalf)
+              rope_row_half<kPT, kPH, 0, 8>(p, sTabC, sTabS, sQ + uint32_t(b * kQTileBytes + rt * 128), kQHalfBytes,
+                                            uint32_t(rt & 7), pt, ph, pw);
+            else
+              rope_row<kPT, kPH, 0, 16>(p, sTabC, sTabS, sQ + uint32_t(b * kQTileBytes + rt * 128), kQHalfBytes,
+                                        uint32_t(rt & 7), pt, ph, pw);
           }
         }
       }
@@ -660,10 +742,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             int pt, ph, pw;
             row_positions(p, row, s.k_t0, pt, ph, pw);
             const uint32_t ra = sK + st * kKStageBytes + uint32_t(r * 128);
-            if (rt < 64)
+            if (kHalf) {
+              // rotate-half: chunk pairs 0-3 / 4-7 (both 64-column halves)
+              if (rt < 64)
+                rope_row_half<kPT, kPH, 0, 4>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
+              else
+                rope_row_half<kPT, kPH, 4, 4>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
+            } else if (rt < 64) {
               rope_row<kPT, kPH, 0, 8>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
-            else
+            } else {
               rope_row<kPT, kPH, 8, 8>(p, sTabC, sTabS, ra, kKHalfBytes, uint32_t(r & 7), pt, ph, pw);
+            }
           }
         }
         ptx::fence_proxy_async_smem();
@@ -920,9 +1009,17 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __g
 
 // Launch shape of the attention kernel (attributes set, cluster of 2) and the
 // number of clusters that fit on the current device at once.
-static rkv_status attn_launch_shape(bool default_split, cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr,
+// Kernel instantiation: the pages' 22/21/21 adjacent-pair split gets a
+// compile-time axis map; other splits and the rotate-half layout read it
+// from the parameters.
+static void (*attn_kernel_for(bool default_split, bool half))(Params) {
+  if (half) return attn_fwd_kernel<0, 0, true>;
+  return default_split ? attn_fwd_kernel<22, 21, false> : attn_fwd_kernel<0, 0, false>;
+}
+
+static rkv_status attn_launch_shape(bool default_split, bool half, cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr,
                                     const void*& kern_ptr, int& max_clusters) {
-  auto kern = default_split ? attn_fwd_kernel<22, 21> : attn_fwd_kernel<0, 0>;
+  auto kern = attn_kernel_for(default_split, half);
   kern_ptr = reinterpret_cast<const void*>(kern);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
@@ -967,7 +1064,7 @@ extern "C" size_t attn_fwd_varlen_workspace_size(const rkv_attn_seq*, int32_t, i
   cudaLaunchAttribute attr[1];
   const void* kern = nullptr;
   int clusters = 0;
-  if (attn_launch_shape(true, cfg, attr, kern, clusters) != RKV_OK) {
+  if (attn_launch_shape(true, false, cfg, attr, kern, clusters) != RKV_OK) {
     clear_error();
     return kWorkspaceBytes;
   }
@@ -1102,7 +1199,9 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   p.F = uint32_t(F);
   p.div_F = make_fastdiv(uint32_t(F));
   p.div_W = make_fastdiv(uint32_t(rope->grid_w));
-  p.log2_theta = log2(double(rope->theta));
+  p.log2_theta[0] = log2(double(rope->theta));
+  p.log2_theta[1] = log2(double(rope->theta_h != 0.0f ? rope->theta_h : rope->theta));
+  p.log2_theta[2] = log2(double(rope->theta_w != 0.0f ? rope->theta_w : rope->theta));
   p.status = static_cast<int32_t*>(workspace);
   p.timeout_ns = 2000000000ull;
 
@@ -1113,7 +1212,8 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   cudaLaunchAttribute attr[1];
   const void* kern = nullptr;
   int max_clusters = 0;
-  if ((st = attn_launch_shape(default_split, cfg, attr, kern, max_clusters)) != RKV_OK) return st;
+  const bool half = rope->layout == RKV_ROPE_HALF;
+  if ((st = attn_launch_shape(default_split, half, cfg, attr, kern, max_clusters)) != RKV_OK) return st;
   cfg.stream = cs;
 
   // tail split: the last n_split units run as two half-units each when the
@@ -1159,8 +1259,7 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
   // one CTA pair per pair of SMs that can hold it (persistent)
   cfg.gridDim = dim3(uint32_t(2 * std::min<int64_t>(p.total_units, max_clusters)));
-  e = default_split ? cudaLaunchKernelEx(&cfg, attn_fwd_kernel<22, 21>, p)
-                    : cudaLaunchKernelEx(&cfg, attn_fwd_kernel<0, 0>, p);
+  e = cudaLaunchKernelEx(&cfg, attn_kernel_for(default_split, half), p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   if (n_split > 0) {

@@ -32,13 +32,14 @@ struct RopeArgs {
   int32_t ring_head, ring_slots;
   uint32_t L;
   uint32_t cpr;            // 16-byte chunks per row = H * 16
+  uint32_t cph;            // rotate-half chunk pairs per row = H * 8
   uint32_t rows_per_cta;
   uint32_t F;              // tokens per frame
   int32_t t0;
   int32_t grid_h, grid_w;
   int32_t pt, ph, pw;      // rotary pairs per axis
-  double log2_theta;
-  FastDiv div_F, div_W, div_cpr;
+  double log2_theta[3];    // per axis t, h, w
+  FastDiv div_F, div_W, div_cpr, div_cph;
 };
 
 // threads per CTA: the standalone op runs one 1024-thread CTA per SM (each
@@ -113,10 +114,34 @@ __device__ __forceinline__ void copy_rows_to_ring(const RopeArgs& a, uint32_t r0
   }
 }
 
+// Rotate the 8 rotary pairs (element e of chunk A, element e of chunk B),
+// e = 0..7, of the rotate-half layout; pair index of element e is p0 + e.
+template <typename TabIdx>
+__device__ __forceinline__ void rotate_half_chunks(uint4& A, uint4& B, int32_t p0, const TabEntry* tab,
+                                                   TabIdx tab_idx) {
+  uint32_t a4[4] = {A.x, A.y, A.z, A.w}, b4[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float y0[2], y1[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x0 = h ? bf16hi_to_f32(a4[w]) : bf16lo_to_f32(a4[w]);
+      const float x1 = h ? bf16hi_to_f32(b4[w]) : bf16lo_to_f32(b4[w]);
+      rotate_pair(x0, x1, tab[tab_idx(p0 + 2 * w + h)], y0[h], y1[h]);
+    }
+    a4[w] = pack_bf16x2(y0[0], y0[1]);
+    b4[w] = pack_bf16x2(y1[0], y1[1]);
+  }
+  A = make_uint4(a4[0], a4[1], a4[2], a4[3]);
+  B = make_uint4(b4[0], b4[1], b4[2], b4[3]);
+}
+
 // kRing = false: rotate rows of x into rows of y (rope3d_apply).
 // kRing = true: blockIdx.y = 0 rotates x (K) into ring slots of y, blockIdx.y
 // = 1 copies x2 (V) into ring slots of y2 (kvcache_ring_update_rope).
-template <bool kRing>
+// kHalf: rotate-half layout (pair j = elements j and j + 64 of a head, i.e.
+// element e of chunk c and of chunk c + 8); else adjacent pairs (2j, 2j+1).
+template <bool kRing, bool kHalf>
 __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const RopeArgs a) {
   constexpr int kRopeThreads = rope_threads<kRing>();
   extern __shared__ float4 tab_raw[];
@@ -162,7 +187,8 @@ __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const Rop
       pos = w_lo + ww;
       if (pos >= a.grid_w) pos -= a.grid_w;
     }
-    const double ang = double(pos) * exp2(-(double(i) / double(n)) * a.log2_theta);
+    const int axis = e < base_h ? 0 : (e < base_w ? 1 : 2);
+    const double ang = double(pos) * exp2(-(double(i) / double(n)) * a.log2_theta[axis]);
     double s, c;
     sincos(ang, &s, &c);
     TabEntry t;
@@ -173,6 +199,49 @@ __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const Rop
     tab[e] = t;
   }
   __syncthreads();
+
+  if (kHalf) {
+    // units of work: chunk pairs (c, c + 8) of a head, 8 per head
+    const uint32_t p_begin = r0 * a.cph, p_end = r1 * a.cph;
+    for (uint32_t base = p_begin + threadIdx.x; base < p_end; base += kRopeThreads * kRopeUnroll) {
+      uint4 va[kRopeUnroll], vb[kRopeUnroll];
+      uint32_t row[kRopeUnroll], ca[kRopeUnroll];
+#pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        const uint32_t pi = base + u * kRopeThreads;
+        if (pi < p_end) {
+          row[u] = fdiv(pi, a.div_cph);
+          const uint32_t wp = pi - row[u] * a.cph;          // head * 8 + c
+          ca[u] = (wp >> 3) * 16u + (wp & 7u);               // chunk c of the head; its partner is ca + 8
+          const uint8_t* src = a.x + int64_t(row[u]) * a.x_stride_bytes;
+          va[u] = *reinterpret_cast<const uint4*>(src + uint64_t(ca[u]) * 16u);
+          vb[u] = *reinterpret_cast<const uint4*>(src + uint64_t(ca[u] + 8u) * 16u);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        const uint32_t pi = base + u * kRopeThreads;
+        if (pi >= p_end) continue;
+        const uint32_t r = row[u];
+        const uint32_t f = fdiv(r, a.div_F);
+        const uint32_t in_f = r - f * a.F;
+        const uint32_t hh = fdiv(in_f, a.div_W);
+        const uint32_t ww = in_f - hh * uint32_t(a.grid_w);
+        int32_t wi_off = int32_t(ww) - w_lo;
+        if (wi_off < 0) wi_off += a.grid_w;
+        const int32_t ti = int32_t(f - f_lo) * a.pt;
+        const int32_t hi = base_h + (int32_t(hh) - h_lo) * a.ph - a.pt;
+        const int32_t wi = base_w + wi_off * a.pw - a.pt - a.ph;
+        const int32_t pt = a.pt, pth = a.pt + a.ph;
+        rotate_half_chunks(va[u], vb[u], int32_t(ca[u] & 7u) * 8, tab, [&](int32_t p) {
+          return p < pt ? ti + p : (p < pth ? hi + p : wi + p);
+        });
+        *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, ca[u])) = va[u];
+        *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, ca[u] + 8u)) = vb[u];
+      }
+    }
+    return;
+  }
 
   const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
   for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
@@ -234,13 +303,19 @@ rkv_status check_rope(const rkv_rope3d* rope, int32_t D) {
   if (rope->pairs_t + rope->pairs_h + rope->pairs_w != D / 2)
     return fail(RKV_ERR_INVALID_ARG, "pairs_t+pairs_h+pairs_w must equal D/2");
   if (!(rope->theta > 1.0f) || !isfinite(rope->theta)) return fail(RKV_ERR_INVALID_ARG, "theta must be finite and > 1");
+  const float th[2] = {rope->theta_h, rope->theta_w};
+  for (int i = 0; i < 2; ++i)
+    if (th[i] != 0.0f && (!(th[i] > 1.0f) || !isfinite(th[i])))
+      return fail(RKV_ERR_INVALID_ARG, "theta_h / theta_w must be 0 (= theta) or finite and > 1");
+  if (rope->layout != RKV_ROPE_ADJACENT && rope->layout != RKV_ROPE_HALF)
+    return fail(RKV_ERR_INVALID_ARG, "rope layout must be RKV_ROPE_ADJACENT or RKV_ROPE_HALF");
   return RKV_OK;
 }
 
 // Fill the rotation part of RopeArgs, pick rows per CTA under the table
 // budget and launch (ring mode: two CTA rows, K rotated and V copied).
-template <bool kRing>
-static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
+template <bool kRing, bool kHalf>
+static rkv_status launch_rope_shape(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
                               cudaStream_t stream) {
   a.L = uint32_t(L);
   a.cpr = uint32_t(H) * 16u;
@@ -251,7 +326,11 @@ static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, con
   a.pt = rope->pairs_t;
   a.ph = rope->pairs_h;
   a.pw = rope->pairs_w;
-  a.log2_theta = log2(double(rope->theta));
+  a.log2_theta[0] = log2(double(rope->theta));
+  a.log2_theta[1] = log2(double(rope->theta_h != 0.0f ? rope->theta_h : rope->theta));
+  a.log2_theta[2] = log2(double(rope->theta_w != 0.0f ? rope->theta_w : rope->theta));
+  a.cph = uint32_t(H) * 8u;
+  a.div_cph = make_fastdiv(a.cph);
   a.div_F = make_fastdiv(a.F);
   a.div_W = make_fastdiv(uint32_t(rope->grid_w));
   a.div_cpr = make_fastdiv(a.cpr);
@@ -270,15 +349,22 @@ static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, con
   const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing, kHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kRopeMaxEntries * int(sizeof(TabEntry)));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
     attr_set = true;
   }
-  rope3d_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
+  rope3d_kernel<kRing, kHalf><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
   return RKV_OK;
+}
+
+template <bool kRing>
+static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
+                              cudaStream_t stream) {
+  return rope->layout == RKV_ROPE_HALF ? launch_rope_shape<kRing, true>(a, L, H, t0, rope, stream)
+                                       : launch_rope_shape<kRing, false>(a, L, H, t0, rope, stream);
 }
 
 }  // namespace rkv

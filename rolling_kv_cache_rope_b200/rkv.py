@@ -30,7 +30,11 @@ STATUS_NAMES = {0: "RKV_OK", 1: "RKV_ERR_INVALID_ARG", 2: "RKV_ERR_UNSUPPORTED",
 
 class rkv_rope3d(ctypes.Structure):
     _fields_ = [("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32), ("pairs_t", ctypes.c_int32),
-                ("pairs_h", ctypes.c_int32), ("pairs_w", ctypes.c_int32), ("theta", ctypes.c_float)]
+                ("pairs_h", ctypes.c_int32), ("pairs_w", ctypes.c_int32), ("theta", ctypes.c_float),
+                ("theta_h", ctypes.c_float), ("theta_w", ctypes.c_float), ("layout", ctypes.c_int32)]
+
+
+RKV_ROPE_ADJACENT, RKV_ROPE_HALF = 0, 1
 
 
 class rkv_attn_seq(ctypes.Structure):
@@ -96,8 +100,14 @@ def _check(status):
         raise RkvError(status, rkv_last_error_string())
 
 
-def make_rope(grid_h, grid_w, pairs=(22, 21, 21), theta=10000.0):
-    return rkv_rope3d(int(grid_h), int(grid_w), int(pairs[0]), int(pairs[1]), int(pairs[2]), float(theta))
+def make_rope(grid_h, grid_w, pairs=(22, 21, 21), theta=10000.0, layout="adjacent"):
+    """RoPE parameters.  ``theta``: one frequency base or a (t, h, w) triple;
+    ``layout``: "adjacent" (pairs 2j, 2j+1) or "half" (pairs j, j + D/2)."""
+    th = tuple(float(v) for v in theta) if isinstance(theta, (tuple, list)) else (float(theta),) * 3
+    if layout not in ("adjacent", "half"):
+        raise ValueError("layout must be 'adjacent' or 'half'")
+    return rkv_rope3d(int(grid_h), int(grid_w), int(pairs[0]), int(pairs[1]), int(pairs[2]), th[0], th[1], th[2],
+                      RKV_ROPE_HALF if layout == "half" else RKV_ROPE_ADJACENT)
 
 
 def _stream(stream):

@@ -126,6 +126,26 @@ def test_rope_rejects(rkv, args, frag):
     assert frag in rkv.rkv_last_error_string()
 
 
+def test_rope_rejects_bad_layout_and_axis_theta(rkv):
+    lib = rkv.lib()
+    for kw in ({"layout": 2}, {"theta_h": 0.5}, {"theta_w": float("inf")}):
+        r = rope(rkv)
+        for k, v in kw.items():
+            setattr(r, k, v)
+        st = lib.rope3d_apply(fake(0x1000), fake(0x90000000), 72, 2, 128, 256, 256, 0, ctypes.byref(r), None)
+        assert st == rkv.RKV_ERR_INVALID_ARG, kw
+        assert ("layout" in rkv.rkv_last_error_string()) or ("theta" in rkv.rkv_last_error_string())
+
+
+def test_make_rope_variants(rkv):
+    r = rkv.make_rope(4, 6, theta=(100.0, 200.0, 300.0), layout="half")
+    assert (r.theta, r.theta_h, r.theta_w, r.layout) == (100.0, 200.0, 300.0, rkv.RKV_ROPE_HALF)
+    d = rkv.make_rope(4, 6)
+    assert (d.theta, d.theta_h, d.theta_w, d.layout) == (10000.0, 10000.0, 10000.0, rkv.RKV_ROPE_ADJACENT)
+    with pytest.raises(ValueError):
+        rkv.make_rope(4, 6, layout="interleaved")
+
+
 def test_rope_zero_rows_is_a_noop(rkv):
     r = rope(rkv)
     assert rkv.lib().rope3d_apply(None, None, 0, 2, 128, 256, 256, 0, ctypes.byref(r), None) == rkv.RKV_OK
