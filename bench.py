@@ -375,6 +375,27 @@ def run_ours(args):
     two_pass_flops = 4.0 * D * H * (visible_pairs(LQ // F, LK // F - LQ // F, LK // F) + visible_pairs(5, 16, LK // F))
     two_pass_ms = time_attn(two_pass)
 
+    # the other RoPE reading: rotate-half pairs, per-axis frequency bases
+    rope_half = rkv.make_rope(GRID_H, GRID_W, theta=(10000.0, 10000.0, 10000.0), layout="half")
+    half_attn = rkv.AttnSeq(t["q"], t["k"], t["v"], o, q_t0=Q_T0, k_t0=K_T0)
+    for _ in range(3):
+        rkv.attn_fwd_varlen([half_attn], rope_half, workspace=ws)
+    hv = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(5)]
+    yq, yk = torch.empty_like(t["q"]), torch.empty_like(t["k"])
+    torch.cuda.synchronize()
+    for i in range(5):
+        hv[i][0].record(stream)
+        rkv.attn_fwd_varlen([half_attn], rope_half, workspace=ws)
+        hv[i][1].record(stream)
+        rkv.rope3d_apply(t["q"], yq, t0=Q_T0, rope=rope_half)
+        rkv.rope3d_apply(t["k"], yk, t0=K_T0, rope=rope_half)
+        hv[i][2].record(stream)
+    torch.cuda.synchronize()
+    rkv.rkv_attn_status(ws)
+    half_attn_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in hv)
+    half_rope_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in hv)
+    del yq, yk
+
     # kernels per step: attention, the merge of split tail units when the
     # persistent grid's last wave is at most half full (same rule as the
     # library, one CTA pair per two SMs), and the ring update
@@ -417,6 +438,10 @@ def run_ours(args):
                          "avg_ms": two_pass_ms, "useful_flops": two_pass_flops,
                          "what": "one launch: denoise 23,400 + cache-update 7,800 queries over 32,760 keys, "
                                  "frame-block-causal (3 frames), RoPE on Q and K; visible pairs only"},
+            "rotate_half": {"attention": ATTN_FLOPS / (half_attn_ms * 1e-3) / 1e12, "attention_unit": "TFLOP/s",
+                            "rope3d": ROPE_BYTES / (half_rope_ms * 1e-3) / 1e9, "rope3d_unit": "GB/s",
+                            "what": "RKV_ROPE_HALF layout (pairs j, j + 64): fused attention of the step and "
+                                    "standalone RoPE of its Q and K"},
             "kv_update_rope": {"value": RING_BYTES / (ring_rope_ms * 1e-3) / 1e9, "unit": "GB/s",
                                "avg_us": ring_rope_ms * 1e3, "bytes_per_call": RING_BYTES,
                                "what": "kvcache_ring_update_rope: 5 raw-K frames rotated into the ring + 5 V frames",

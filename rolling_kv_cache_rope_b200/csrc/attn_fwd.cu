@@ -1009,11 +1009,10 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __g
 
 // Launch shape of the attention kernel (attributes set, cluster of 2) and the
 // number of clusters that fit on the current device at once.
-// Kernel instantiation: the pages' 22/21/21 adjacent-pair split gets a
-// compile-time axis map; other splits and the rotate-half layout read it
-// from the parameters.
+// Kernel instantiation: the pages' 22/21/21 split gets a compile-time axis
+// map (either pair layout); other splits read it from the parameters.
 static void (*attn_kernel_for(bool default_split, bool half))(Params) {
-  if (half) return attn_fwd_kernel<0, 0, true>;
+  if (half) return default_split ? attn_fwd_kernel<22, 21, true> : attn_fwd_kernel<0, 0, true>;
   return default_split ? attn_fwd_kernel<22, 21, false> : attn_fwd_kernel<0, 0, false>;
 }
 
