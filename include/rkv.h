@@ -230,8 +230,22 @@ rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int
  * Video Generation on Trainium Chips", item 6 "Neuron Kernel Interface").
  *
  * Layout: k and v are device bf16 [slots][tokens_per_frame][H][D], contiguous.
- * `head` = slot the next frame goes to; `count` = valid frames (0..slots).
- * Logical frame j (0 = oldest valid) lives in slot (head - count + j) mod slots.
+ * `count` = valid frames (0..slots).
+ *
+ * Pinned prefix (optional; the pages describe only the sliding window; this
+ * is the common variant that keeps a stream's first frames, "attention
+ * sinks", out of eviction): the first `pinned` slots (0 <= pinned < slots)
+ * take the first `pinned` frames ever inserted and are never overwritten;
+ * every later frame rolls through slots [pinned, slots).  pinned = 0 is the
+ * plain ring.
+ *
+ * `head` = the slot of [pinned, slots) the next rolling frame goes to; a new
+ * ring starts with head = pinned, count = 0, and head stays at pinned until
+ * the pinned slots are all filled.  Logical frame j (0 = oldest valid) lives
+ * in slot j when j < pinned, else in slot
+ *   pinned + (head - pinned - (count - pinned) + (j - pinned)) mod (slots - pinned)
+ * which for pinned = 0 is (head - count + j) mod slots.  A ring filled from
+ * empty has its valid frames in the slot prefix [0, count), in any state.
  */
 typedef struct {
   void* k;
@@ -240,8 +254,9 @@ typedef struct {
   int32_t tokens_per_frame;
   int32_t H;
   int32_t D;
-  int32_t head;  /* updated by kvcache_ring_update (host side) */
-  int32_t count; /* updated by kvcache_ring_update (host side) */
+  int32_t head;   /* updated by kvcache_ring_update (host side) */
+  int32_t count;  /* updated by kvcache_ring_update (host side) */
+  int32_t pinned; /* slots of the pinned prefix; fixed for the ring's life */
 } rkv_ring;
 
 /*
@@ -250,13 +265,20 @@ typedef struct {
  *   ring           caller's ring; head/count are updated on success
  *   k_new, v_new   device bf16 [n_frames * tokens_per_frame][H][D] with row
  *                  stride new_row_stride (elements); must not overlap the ring
- *   n_frames       0..slots (0 = no-op)
+ *   n_frames       0..capacity (0 = no-op), capacity = the free pinned slots
+ *                  max(0, pinned - count) plus the rolling slots
+ *                  slots - pinned (= slots without a pinned prefix)
  *   n_evicted      optional out: frames dropped = max(0, count + n - slots)
- * Frame i goes to slot (head + i) mod slots; then head = (head + n) mod slots,
- * count = min(slots, count + n).  Evicted frames are overwritten, not
- * cleared: no bytes move for eviction.
- * Errors: RKV_ERR_INVALID_ARG (n_frames > slots or < 0, null pointers,
- * head/count out of range, D != 128, misalignment, overlap).
+ * The first p = min(n, max(0, pinned - count)) frames go to slots count,
+ * count + 1, ...; frame i >= p goes to slot
+ * pinned + (head - pinned + i - p) mod (slots - pinned).  Then
+ * head = pinned + (head - pinned + n - p) mod (slots - pinned) and
+ * count = min(slots, count + n).  Without a pinned prefix frame i goes to
+ * slot (head + i) mod slots.  Evicted frames are overwritten, not cleared:
+ * no bytes move for eviction.
+ * Errors: RKV_ERR_INVALID_ARG (n_frames above capacity or < 0, null
+ * pointers, pinned/head/count out of range or inconsistent, D != 128,
+ * misalignment, overlap).
  */
 rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_new,
                                int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,

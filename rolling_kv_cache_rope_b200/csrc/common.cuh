@@ -22,6 +22,23 @@ rkv_status check_ring_insert(const rkv_ring* ring, const void* k_new, const void
                              int32_t n_frames);                     // ring_update.cu
 void ring_advance(rkv_ring* ring, int32_t n_frames, int32_t* n_evicted);  // head, count, evicted
 
+// Where the frames of one insert land.  The first n_pin frames fill the free
+// slots of the pinned prefix from pin_base on; the rest roll through the
+// region [end - len, end) from head on, wrapping once at most (an insert
+// carries at most len rolling frames).  Without a pinned prefix n_pin = 0 and
+// the region is the whole ring.
+struct RingPlan {
+  int32_t n_pin, pin_base, head, end, len;
+};
+RingPlan ring_plan(const rkv_ring* ring);  // ring_update.cu; for a checked ring
+
+__host__ __device__ __forceinline__ int32_t ring_dst_slot(const RingPlan& p, uint32_t frame) {
+  const int32_t f = int32_t(frame);
+  if (f < p.n_pin) return p.pin_base + f;
+  const int32_t s = p.head + (f - p.n_pin);
+  return s >= p.end ? s - p.len : s;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Byte ranges [a, a+na) and [b, b+nb) overlap.

@@ -26,7 +26,7 @@ struct RingCopyArgs {
   uint32_t row_vecs;      // row_bytes / 16
   uint32_t total_vecs;    // n_frames * tokens_per_frame * row_vecs
   uint32_t F;             // tokens per frame
-  int32_t head, slots;
+  RingPlan plan;          // destination slot of each inserted frame
   FastDiv div_row_vecs, div_F;
 };
 
@@ -51,8 +51,7 @@ __global__ void __launch_bounds__(kRingThreads) ring_copy_kernel(const RingCopyA
         const uint32_t c = v - row * a.row_vecs;
         const uint32_t frame = fdiv(row, a.div_F);
         const uint32_t rr = row - frame * a.F;
-        int32_t slot = a.head + int32_t(frame);
-        if (slot >= a.slots) slot -= a.slots;
+        const int32_t slot = ring_dst_slot(a.plan, frame);
         val[u] = __ldcs(reinterpret_cast<const uint4*>(src + int64_t(row) * a.src_row_stride_bytes +
                                                         uint64_t(c) * 16u));
         out[u] = dst + uint64_t(slot) * a.frame_bytes + uint64_t(rr) * a.row_bytes + uint64_t(c) * 16u;
@@ -76,9 +75,14 @@ rkv_status check_ring(const rkv_ring* r) {
   if (r->slots < 1 || r->tokens_per_frame < 1 || r->H < 1)
     return fail(RKV_ERR_INVALID_ARG, "ring slots/tokens_per_frame/H must be >= 1");
   if (r->D != 128) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", r->D);
-  if (r->head < 0 || r->head >= r->slots) return fail(RKV_ERR_INVALID_ARG, "ring head %d out of range", r->head);
+  if (r->pinned < 0 || r->pinned >= r->slots)
+    return fail(RKV_ERR_INVALID_ARG, "ring pinned %d must be in [0, slots=%d)", r->pinned, r->slots);
+  if (r->head < r->pinned || r->head >= r->slots)
+    return fail(RKV_ERR_INVALID_ARG, "ring head %d out of range [pinned, slots)", r->head);
   if (r->count < 0 || r->count > r->slots)
     return fail(RKV_ERR_INVALID_ARG, "ring count %d out of range", r->count);
+  if (r->count < r->pinned && r->head != r->pinned)
+    return fail(RKV_ERR_INVALID_ARG, "ring head must equal pinned until the pinned frames are all in");
   if (!aligned16(r->k) || !aligned16(r->v)) return fail(RKV_ERR_INVALID_ARG, "ring buffers must be 16-byte aligned");
   const uint64_t bytes = uint64_t(r->slots) * r->tokens_per_frame * r->H * r->D * 2;
   if (overlaps(r->k, bytes, r->v, bytes)) return fail(RKV_ERR_INVALID_ARG, "ring k and v buffers overlap");
@@ -87,8 +91,11 @@ rkv_status check_ring(const rkv_ring* r) {
 
 rkv_status check_ring_insert(const rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
                              int32_t n_frames) {
-  if (n_frames < 0 || n_frames > ring->slots)
-    return fail(RKV_ERR_INVALID_ARG, "n_frames %d must be in [0, slots=%d]", n_frames, ring->slots);
+  const int32_t free_pinned = ring->count < ring->pinned ? ring->pinned - ring->count : 0;
+  const int32_t capacity = free_pinned + (ring->slots - ring->pinned);
+  if (n_frames < 0 || n_frames > capacity)
+    return fail(RKV_ERR_INVALID_ARG, "n_frames %d must be in [0, %d] (free pinned slots + rolling slots)", n_frames,
+                capacity);
   if (n_frames == 0) return RKV_OK;
   const int64_t row_elems = int64_t(ring->H) * ring->D;
   if (!k_new || !v_new) return fail(RKV_ERR_INVALID_ARG, "k_new/v_new is NULL");
@@ -106,10 +113,24 @@ rkv_status check_ring_insert(const rkv_ring* ring, const void* k_new, const void
   return RKV_OK;
 }
 
+RingPlan ring_plan(const rkv_ring* ring) {
+  RingPlan p;
+  p.pin_base = ring->count;
+  p.n_pin = ring->count < ring->pinned ? ring->pinned - ring->count : 0;
+  p.head = ring->head;
+  p.end = ring->slots;
+  p.len = ring->slots - ring->pinned;
+  return p;
+}
+
 void ring_advance(rkv_ring* ring, int32_t n_frames, int32_t* n_evicted) {
-  const int32_t evicted = ring->count + n_frames > ring->slots ? ring->count + n_frames - ring->slots : 0;
-  ring->head = (ring->head + n_frames) % ring->slots;
-  ring->count = ring->count + n_frames < ring->slots ? ring->count + n_frames : ring->slots;
+  const RingPlan p = ring_plan(ring);
+  const int32_t pinned_in = n_frames < p.n_pin ? n_frames : p.n_pin;
+  const int32_t rolling = n_frames - pinned_in;
+  const int32_t count = ring->count + pinned_in;
+  const int32_t evicted = count + rolling > ring->slots ? count + rolling - ring->slots : 0;
+  ring->head = ring->pinned + (ring->head - ring->pinned + rolling) % p.len;
+  ring->count = count + rolling < ring->slots ? count + rolling : ring->slots;
   if (n_evicted) *n_evicted = evicted;
 }
 
@@ -118,13 +139,17 @@ void ring_advance(rkv_ring* ring, int32_t n_frames, int32_t* n_evicted) {
 using namespace rkv;
 
 extern "C" int32_t rkv_ring_slot(const rkv_ring* ring, int32_t j) {
-  if (!ring || ring->slots < 1 || ring->count < 0 || ring->count > ring->slots || ring->head < 0 ||
-      ring->head >= ring->slots)
+  if (!ring || ring->slots < 1 || ring->pinned < 0 || ring->pinned >= ring->slots || ring->count < 0 ||
+      ring->count > ring->slots || ring->head < ring->pinned || ring->head >= ring->slots)
     return -1;
   if (j < 0 || j >= ring->count) return -1;
-  int64_t s = (int64_t(ring->head) - ring->count + j) % ring->slots;
-  if (s < 0) s += ring->slots;
-  return int32_t(s);
+  const int32_t P = ring->pinned;
+  if (j < P) return j;
+  // rolling frame j - P of count - P, the newest one in slot head - 1
+  const int32_t len = ring->slots - P;
+  int64_t s = (int64_t(ring->head - P) - (ring->count - P) + (j - P)) % len;
+  if (s < 0) s += len;
+  return int32_t(P + s);
 }
 
 extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_new,
@@ -149,8 +174,7 @@ extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, con
     a.frame_bytes = uint64_t(ring->tokens_per_frame) * a.row_bytes;
     a.total_vecs = uint32_t(total_vecs);
     a.F = uint32_t(ring->tokens_per_frame);
-    a.head = ring->head;
-    a.slots = ring->slots;
+    a.plan = ring_plan(ring);
     a.div_row_vecs = make_fastdiv(a.row_vecs);
     a.div_F = make_fastdiv(a.F);
     const uint64_t per_block = uint64_t(kRingThreads) * kRingUnroll;

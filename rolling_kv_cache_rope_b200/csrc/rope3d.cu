@@ -29,7 +29,7 @@ struct RopeArgs {
   uint8_t* y2;
   int64_t x_stride_bytes, y_stride_bytes;
   uint64_t slot_bytes;     // ring mode: bytes of one ring slot (one frame)
-  int32_t ring_head, ring_slots;
+  RingPlan ring;           // ring mode: destination slot of each frame
   uint32_t L;
   uint32_t cpr;            // 16-byte chunks per row = H * 16
   uint32_t cph;            // rotate-half chunk pairs per row = H * 8
@@ -76,14 +76,13 @@ __device__ __forceinline__ void rotate_pair(float x0, float x1, const TabEntry& 
 }
 
 // Address of 16-byte chunk `within` of row r (frame f, row in_f of that
-// frame) in the destination: a strided row, or the row's place in ring slot
-// (head + f) mod slots.
+// frame) in the destination: a strided row, or the row's place in the ring
+// slot that frame f of the insert goes to.
 template <bool kRing>
 __device__ __forceinline__ uint8_t* dst_chunk(const RopeArgs& a, uint8_t* base, uint32_t r, uint32_t f, uint32_t in_f,
                                               uint32_t within) {
   if (kRing) {
-    int32_t slot = a.ring_head + int32_t(f);
-    if (slot >= a.ring_slots) slot -= a.ring_slots;
+    const int32_t slot = ring_dst_slot(a.ring, f);
     return base + uint64_t(slot) * a.slot_bytes + (uint64_t(in_f) * a.cpr + within) * 16u;
   }
   return base + int64_t(r) * a.y_stride_bytes + uint64_t(within) * 16u;
@@ -424,8 +423,7 @@ extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new
     a.x_stride_bytes = new_row_stride * 2;
     a.y_stride_bytes = int64_t(ring->H) * ring->D * 2;
     a.slot_bytes = uint64_t(ring->tokens_per_frame) * ring->H * ring->D * 2;
-    a.ring_head = ring->head;
-    a.ring_slots = ring->slots;
+    a.ring = ring_plan(ring);
     st = launch_rope<true>(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope,
                            static_cast<cudaStream_t>(stream));
     if (st != RKV_OK) return st;

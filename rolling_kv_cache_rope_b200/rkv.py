@@ -48,7 +48,7 @@ class rkv_attn_seq(ctypes.Structure):
 class rkv_ring(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("slots", ctypes.c_int32),
                 ("tokens_per_frame", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
-                ("head", ctypes.c_int32), ("count", ctypes.c_int32)]
+                ("head", ctypes.c_int32), ("count", ctypes.c_int32), ("pinned", ctypes.c_int32)]
 
 
 _c = ctypes
@@ -190,14 +190,15 @@ def rkv_attn_status(workspace, stream=None):
 
 class KVRing:
     """A per-layer ring of frame slots for K and V (device bf16
-    [slots][tokens_per_frame][H][D] each) plus its head/count state."""
+    [slots][tokens_per_frame][H][D] each) plus its head/count state; the
+    first ``pinned`` slots keep the first frames ever inserted."""
 
-    def __init__(self, slots, tokens_per_frame, H, D=128, device="cuda", k=None, v=None):
+    def __init__(self, slots, tokens_per_frame, H, D=128, device="cuda", k=None, v=None, pinned=0):
         import torch
         shape = (slots, tokens_per_frame, H, D)
         self.k = torch.empty(shape, dtype=torch.bfloat16, device=device) if k is None else k
         self.v = torch.empty(shape, dtype=torch.bfloat16, device=device) if v is None else v
-        self.c = rkv_ring(self.k.data_ptr(), self.v.data_ptr(), slots, tokens_per_frame, H, D, 0, 0)
+        self.c = rkv_ring(self.k.data_ptr(), self.v.data_ptr(), slots, tokens_per_frame, H, D, pinned, 0, pinned)
 
     @property
     def head(self):
@@ -210,6 +211,10 @@ class KVRing:
     @property
     def slots(self):
         return self.c.slots
+
+    @property
+    def pinned(self):
+        return self.c.pinned
 
     def slot(self, j):
         return int(_lib.rkv_ring_slot(ctypes.byref(self.c), int(j)))

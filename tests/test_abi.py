@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -44,8 +45,8 @@ def test_version(rkv):
     assert rkv.rkv_version() >= 100
 
 
-def ring(rkv, slots=5, F=24, H=2, D=128, head=0, count=0, k=0x10000, v=0x20000000):
-    return rkv.rkv_ring(k, v, slots, F, H, D, head, count)
+def ring(rkv, slots=5, F=24, H=2, D=128, head=0, count=0, k=0x10000, v=0x20000000, pinned=0):
+    return rkv.rkv_ring(k, v, slots, F, H, D, head, count, pinned)
 
 
 def test_ring_slot_host_logic(rkv):
@@ -69,6 +70,12 @@ def test_ring_slot_host_logic(rkv):
     (dict(k=0), 1, "NULL"),
     (dict(k=0x10008), 1, "aligned"),
     (dict(v=0x10000), 1, "overlap"),         # k and v buffers overlap
+    (dict(pinned=5), 1, "pinned"),           # pinned must leave a rolling slot
+    (dict(pinned=-1), 1, "pinned"),
+    (dict(pinned=2, head=1, count=5), 1, "head"),   # head inside the pinned prefix
+    (dict(pinned=2, head=3, count=1), 1, "head"),   # rolling before the prefix is full
+    (dict(pinned=2, head=2, count=5), 4, "n_frames"),   # 3 rolling slots, prefix full
+    (dict(pinned=2, head=2, count=1), 5, "n_frames"),   # 1 free pinned + 3 rolling
 ])
 def test_ring_update_rejects(rkv, change, n, frag):
     lib = rkv.lib()
@@ -80,6 +87,23 @@ def test_ring_update_rejects(rkv, change, n, frag):
     assert st == rkv.RKV_ERR_INVALID_ARG
     assert frag in rkv.rkv_last_error_string()
     assert (r.head, r.count) == before and ev.value == -7
+
+
+def test_ring_slot_pinned_matches_oracle(rkv):
+    # slot of every logical frame, in every state a pinned ring passes through
+    from oracle import RingRef
+    lib = rkv.lib()
+    rng = np.random.default_rng(5)
+    for W, P in [(5, 1), (6, 2), (21, 3), (4, 3)]:
+        ref = RingRef(W, P)
+        for _ in range(40):
+            n = int(rng.integers(0, ref.capacity_for_insert() + 1))
+            ref.insert([None] * n)
+            r = ring(rkv, slots=W, head=ref.head, count=ref.count, pinned=P)
+            got = [lib.rkv_ring_slot(ctypes.byref(r), j) for j in range(-1, W + 1)]
+            assert got == [ref.slot_of(j) for j in range(-1, W + 1)], (W, P, ref.head, ref.count)
+    bad = ring(rkv, slots=5, head=1, count=5, pinned=2)
+    assert lib.rkv_ring_slot(ctypes.byref(bad), 0) == -1
 
 
 def test_ring_update_rejects_bad_sources(rkv):
