@@ -276,6 +276,9 @@ typedef struct {
  * count = min(slots, count + n).  Without a pinned prefix frame i goes to
  * slot (head + i) mod slots.  Evicted frames are overwritten, not cleared:
  * no bytes move for eviction.
+ * The copy runs on the TMA bulk-copy engine; each of its waits on a bulk
+ * load is bounded (1 s), after which the kernel stops, sets a per-GPU flag and
+ * the insert is incomplete: rkv_ring_status reads that flag.
  * Errors: RKV_ERR_INVALID_ARG (n_frames above capacity or < 0, null
  * pointers, pinned/head/count out of range or inconsistent, D != 128,
  * misalignment, overlap).
@@ -311,6 +314,14 @@ rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_
 rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
                                     int64_t new_row_stride, int32_t n_frames, int32_t t0,
                                     const rkv_rope3d* rope, int32_t* n_evicted, void* stream);
+
+/*
+ * rkv_ring_status -- synchronise `stream` and report whether a ring insert on
+ * the current GPU gave up on a bounded device-side wait since the last call:
+ * RKV_ERR_TIMEOUT (the flag is then cleared) or RKV_OK.  Errors:
+ * RKV_ERR_CUDA when the flag cannot be read.
+ */
+rkv_status rkv_ring_status(void* stream);
 
 /* Slot of logical frame j (0 = oldest valid), or -1 when j is not a valid
  * frame or the ring is malformed. */

@@ -1,5 +1,5 @@
-// Thin inline-PTX wrappers for the sm_100a features the attention kernel uses:
-// mbarriers (with bounded waits), TMA tensor loads, tcgen05 TMEM allocation,
+// Thin inline-PTX wrappers for the sm_100a features the kernels use:
+// mbarriers (with bounded waits), TMA tensor and bulk copies, tcgen05 TMEM allocation,
 // MMA, commit, loads/stores and the fences that order them.  Written from the
 // PTX ISA's instruction descriptions; no library code is pulled in.
 #pragma once
@@ -152,6 +152,29 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* desc, uint
       "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+
+// ---- bulk copies (untiled TMA) ------------------------------------------------
+// Global -> this CTA's shared memory; completion is signalled on `bar` as
+// transaction bytes.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// Shared memory -> global, tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all of this thread's committed groups are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---- tcgen05: tensor memory ---------------------------------------------------
 // Pair (cta_group::2) forms: both CTAs of a 2-CTA cluster allocate the same

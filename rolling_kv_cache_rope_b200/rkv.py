@@ -68,6 +68,8 @@ _lib.kvcache_ring_update.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_voi
 _lib.kvcache_ring_update_rope.restype = _c.c_int
 _lib.kvcache_ring_update_rope.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
                                           _c.c_int32, _c.POINTER(rkv_rope3d), _c.POINTER(_c.c_int32), _c.c_void_p]
+_lib.rkv_ring_status.restype = _c.c_int
+_lib.rkv_ring_status.argtypes = [_c.c_void_p]
 _lib.rkv_ring_slot.restype = _c.c_int32
 _lib.rkv_ring_slot.argtypes = [_c.POINTER(rkv_ring), _c.c_int32]
 _lib.rkv_last_error_string.restype = _c.c_char_p
@@ -186,6 +188,12 @@ def attn_fwd_varlen(seqs, rope, softmax_scale=None, workspace=None, stream=None)
 def rkv_attn_status(workspace, stream=None):
     """Synchronise and raise RkvError if the last launch on ``workspace`` timed out."""
     _check(_lib.rkv_attn_status(workspace.data_ptr(), _stream(stream)))
+
+
+def rkv_ring_status(stream=None):
+    """Synchronise and raise RkvError if a ring insert on this GPU gave up on
+    a bounded device-side wait since the last call."""
+    _check(_lib.rkv_ring_status(_stream(stream)))
 
 
 class KVRing:

@@ -1,5 +1,9 @@
 """Ring KV-cache update on the GPU vs the ring oracle: bit-exact indices,
-eviction counts and slot contents; guard frames around the ring stay intact."""
+eviction counts and slot contents; guard frames around the ring stay intact;
+no bounded device-side wait of the bulk copy gives up.  Shapes cover the
+ways an insert is cut into bulk-copy pieces: many rows per piece with a
+short last piece, strided source rows (one load per row), and rows wider
+than a piece (each row split across pieces)."""
 
 import numpy as np
 import pytest
@@ -41,6 +45,7 @@ def run_ring(slots, F, H, inserts, seed, stride_mult=1):
         frames = [(kb[i * F:(i + 1) * F], vb[i * F:(i + 1) * F], frame_no + i) for i in range(n)]
         frame_no += n
         ev = rkv.kvcache_ring_update(ring, kd, vd, n)
+        rkv.rkv_ring_status()   # raises if a device-side wait gave up
         ev_ref = ref.insert(frames)
         assert ev == ev_ref
         assert (ring.head, ring.count) == (ref.head, ref.count)
@@ -90,3 +95,15 @@ def test_random_insert_sizes():
 
 def test_single_slot_ring():
     run_ring(1, 24, 2, [1, 1, 0, 1], seed=901)
+
+
+def test_one_head_many_rows_per_piece():
+    # 256-byte rows: 128 rows per piece, 300-row frames end in a short piece
+    run_ring(4, 300, 1, [3, 2, 4], seed=902)
+    run_ring(3, 300, 1, [2, 3], seed=903, stride_mult=2)
+
+
+def test_rows_wider_than_a_piece():
+    # 160 heads: 40 KB rows, each split into a 32 KB and an 8 KB piece
+    run_ring(4, 6, 160, [3, 2, 4], seed=904)
+    run_ring(3, 5, 160, [2, 3], seed=905, stride_mult=2)
