@@ -19,110 +19,45 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "ring_bulk.cuh"
 #include "sm100_ptx.cuh"
 
 namespace rkv {
 
-constexpr int kBulkStages = 6;
-constexpr uint32_t kBulkStageBytes = 32768;
 constexpr int kBulkThreads = 32;
-constexpr uint64_t kBulkWaitNs = 1000000000ull;  // 1 s per wait, then give up
 
-// Piece p of an insert: tensor p % 2 (K, V), then frame, then a group of rpp
-// whole rows of that frame (or, when one row exceeds a stage, a chunk of one
-// row: cpr chunks per row).
-struct RingBulkArgs {
-  const uint8_t* src[2];
-  uint8_t* dst[2];
-  uint64_t src_row_stride;  // bytes between source rows
-  uint64_t frame_bytes;     // bytes of one ring slot
-  uint32_t row_bytes;       // H * D * 2
-  uint32_t F;               // rows (tokens) per frame
-  uint32_t rpp;             // rows per piece
-  uint32_t cpr;             // pieces across one row (1 unless a row exceeds a stage)
-  uint32_t chunk;           // bytes of each row a piece covers (row_bytes when cpr = 1)
-  uint32_t ppf;             // pieces per frame = ceil(F / rpp) * cpr
-  uint32_t total;           // pieces of the insert = 2 * n_frames * ppf
-  uint32_t stage_bytes;     // rpp * chunk
-  uint32_t contiguous;      // source rows are back to back (one load per piece)
-  RingPlan plan;            // destination slot of each frame
-  int32_t* timeout_flag;    // set to 1 when a wait gives up
-};
-
-struct RingPiece {
-  const uint8_t* src;
-  uint8_t* dst;
-  uint32_t rows, cols;
-};
-
-__device__ __forceinline__ RingPiece ring_piece(const RingBulkArgs& a, uint32_t p) {
-  const uint32_t which = p & 1u, q = p >> 1;
-  const uint32_t frame = q / a.ppf, k = q - frame * a.ppf;
-  const uint32_t rg = k / a.cpr, cc = k - rg * a.cpr;
-  const uint32_t row0 = rg * a.rpp, col0 = cc * a.chunk;
-  RingPiece pc;
-  pc.rows = min(a.rpp, a.F - row0);
-  pc.cols = min(a.chunk, a.row_bytes - col0);
-  const int32_t slot = ring_dst_slot(a.plan, frame);
-  pc.src = a.src[which] + (uint64_t(frame) * a.F + row0) * a.src_row_stride + col0;
-  pc.dst = a.dst[which] + uint64_t(slot) * a.frame_bytes + uint64_t(row0) * a.row_bytes + col0;
-  return pc;
-}
-
+// Piece i of this CTA is staged in slot i % stages, i.e. phase
+// (i / stages) & 1 of that slot's mbarrier.
 __global__ void __launch_bounds__(kBulkThreads, 1) ring_bulk_kernel(const RingBulkArgs a) {
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t full[kBulkStages];
   if (threadIdx.x != 0) return;
-  const uint32_t G = gridDim.x;
-  const uint32_t n = a.total > blockIdx.x ? (a.total - blockIdx.x + G - 1) / G : 0;
-  for (int s = 0; s < kBulkStages; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
-  ptx::fence_mbar_init();
+  const uint32_t n = cta_pieces(a.total, gridDim.x);
   const uint32_t smem0 = ptx::smem_u32(stage_mem);
-
-  // piece i of this CTA is piece blockIdx.x + i * G of the insert, staged in
-  // slot i % kBulkStages (phase i / kBulkStages of that slot's barrier)
-  auto load = [&](uint32_t i) {
-    const RingPiece pc = ring_piece(a, blockIdx.x + i * G);
-    const uint32_t bar = ptx::smem_u32(&full[i % kBulkStages]);
-    const uint32_t dst = smem0 + (i % kBulkStages) * a.stage_bytes;
-    ptx::mbar_expect_tx(bar, pc.rows * pc.cols);
-    if (a.contiguous) {
-      ptx::bulk_load(dst, pc.src, pc.rows * pc.cols, bar);
-    } else {
-      for (uint32_t r = 0; r < pc.rows; ++r) ptx::bulk_load(dst + r * pc.cols, pc.src + r * a.src_row_stride, pc.cols, bar);
-    }
-  };
-  auto wait_full = [&](uint32_t i) {
-    const uint32_t bar = ptx::smem_u32(&full[i % kBulkStages]);
-    const uint32_t parity = (i / kBulkStages) & 1u;
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait(bar, parity))
-      if (ptx::globaltimer_ns() - t0 > kBulkWaitNs) return false;
-    return true;
-  };
-
+  for (uint32_t s = 0; s < a.stages; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+  ptx::fence_mbar_init();
+  auto stage = [&](uint32_t i) { return smem0 + (i % a.stages) * a.stage_bytes; };
+  auto bar = [&](uint32_t i) { return ptx::smem_u32(&full[i % a.stages]); };
   uint32_t issued = 0;
-  for (; issued < n && issued < uint32_t(kBulkStages); ++issued) load(issued);
+  for (; issued < n && issued < a.stages; ++issued) bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued));
   uint32_t i = 0;
   for (; i < n; ++i) {
-    if (!wait_full(i)) {
+    if (!bulk_wait(bar(i), (i / a.stages) & 1u)) {
       atomicExch(a.timeout_flag, 1);
       break;
     }
-    const RingPiece pc = ring_piece(a, blockIdx.x + i * G);
-    ptx::bulk_store(pc.dst, smem0 + (i % kBulkStages) * a.stage_bytes, pc.rows * pc.cols);
-    ptx::bulk_commit();
-    // refill the previous piece's slot once its store has read shared memory
-    // (issued == i - 1 + kBulkStages here)
+    bulk_store_piece(cta_piece(a, i), stage(i));
+    // refill the previous piece's stage once its store has read shared memory
+    // (issued == i - 1 + stages here)
     if (i >= 1 && issued < n) {
       ptx::bulk_wait_read<1>();
-      load(issued++);
+      bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued));
+      ++issued;
     }
   }
   // after a wait gave up: let the loads still in flight land (bounded) before
   // the CTA's shared memory is released
-  for (uint32_t j = i + 1; j < issued; ++j) wait_full(j);
+  for (uint32_t j = i + 1; j < issued; ++j) bulk_wait(bar(j), (j / a.stages) & 1u);
   ptx::bulk_wait_all();
 }
 
@@ -227,35 +162,11 @@ static rkv_status ring_timeout_flag(int32_t** out) {
 static rkv_status launch_ring_bulk(const rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
                                    int32_t n_frames, cudaStream_t stream) {
   RingBulkArgs a;
-  a.src[0] = static_cast<const uint8_t*>(k_new);
-  a.src[1] = static_cast<const uint8_t*>(v_new);
-  a.dst[0] = static_cast<uint8_t*>(ring->k);
-  a.dst[1] = static_cast<uint8_t*>(ring->v);
-  a.row_bytes = uint32_t(int64_t(ring->H) * ring->D * 2);
-  a.src_row_stride = uint64_t(new_row_stride) * 2;
-  a.F = uint32_t(ring->tokens_per_frame);
-  a.frame_bytes = uint64_t(a.F) * a.row_bytes;
-  if (a.row_bytes <= kBulkStageBytes) {
-    a.rpp = kBulkStageBytes / a.row_bytes;
-    if (a.rpp > a.F) a.rpp = a.F;
-    a.cpr = 1;
-    a.chunk = a.row_bytes;
-  } else {
-    a.rpp = 1;
-    a.chunk = kBulkStageBytes;
-    a.cpr = (a.row_bytes + kBulkStageBytes - 1) / kBulkStageBytes;
-  }
-  a.stage_bytes = a.rpp * a.chunk;
-  const uint64_t ppf = uint64_t((a.F + a.rpp - 1) / a.rpp) * a.cpr;
-  const uint64_t total = 2 * uint64_t(n_frames) * ppf;
-  if (total >= (uint64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "insert too large for one launch");
-  a.ppf = uint32_t(ppf);
-  a.total = uint32_t(total);
-  a.contiguous = a.src_row_stride == a.row_bytes ? 1u : 0u;
-  a.plan = ring_plan(ring);
-  rkv_status st = ring_timeout_flag(&a.timeout_flag);
+  rkv_status st = ring_bulk_geometry(ring, k_new, v_new, new_row_stride, n_frames, a);
   if (st != RKV_OK) return st;
-  const int smem = kBulkStages * int(a.stage_bytes);
+  st = ring_timeout_flag(&a.timeout_flag);
+  if (st != RKV_OK) return st;
+  const int smem = int(a.stages * a.stage_bytes);
   cudaError_t e = cudaFuncSetAttribute(ring_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(ring_bulk_kernel)");
   const uint32_t grid = a.total < uint32_t(sm_count()) ? a.total : uint32_t(sm_count());

@@ -54,6 +54,7 @@ def run_pinned(slots, pinned, grid_h, grid_w, H, inserts, seed, rotate):
             ev = rkv.kvcache_ring_update_rope(ring, kd, vd, t, rope, n)
         else:
             ev = rkv.kvcache_ring_update(ring, kd, vd, n)
+        rkv.rkv_ring_status()
         t += n
         assert ev == ref.insert(frames), step
         assert (ring.head, ring.count) == (ref.head, ref.count), step

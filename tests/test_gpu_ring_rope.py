@@ -3,7 +3,9 @@ oracles: every K slot within one bf16 ulp of the correctly rounded fp64
 rotation of the frame it should hold (rotated at that frame's time index);
 V slots, head, count, eviction and slot map bit-exact against RingRef; guard
 frames around the ring untouched.  A consistency check beside the parity
-check: the K slots equal what rope3d_apply writes for the same rows."""
+check: the K slots equal what rope3d_apply writes for the same rows.  Shapes
+include a long w axis and a one-row grid of 4,000 columns, where each CTA's
+cos/sin table holds only the columns its rows reach."""
 
 import numpy as np
 import pytest
@@ -46,6 +48,7 @@ def run_ring_rope(slots, grid_h, grid_w, H, inserts, seed, stride_mult=1, t_star
         kr = kr.reshape(n * F, H * D)
         frames = [(kr[i * F:(i + 1) * F], vb[i * F:(i + 1) * F], t + i) for i in range(n)]
         ev = rkv.kvcache_ring_update_rope(ring, kd, vd, t, rope, n)
+        rkv.rkv_ring_status()   # raises if a device-side wait gave up
         ev_ref = ref.insert(frames)
         # consistency: the standalone call on the same rows
         ky = torch.empty((n * F, H, D), dtype=torch.bfloat16, device="cuda")
@@ -93,6 +96,16 @@ def test_sweep_ring_rope_21_slots_full_schedule():
 
 def test_ring_rope_strided_source_and_late_time():
     run_ring_rope(6, 5, 7, 3, [4, 4, 4], seed=77, stride_mult=3, t_start=1000)
+
+
+def test_ring_rope_wide_grid():
+    # a 4x100 grid: 100 w positions against 4 h positions
+    run_ring_rope(4, 4, 100, 2, [3, 2, 3], seed=78)
+
+
+def test_ring_rope_one_row_grid():
+    # a 1x4000 grid: a table of every position would need 84,000 entries
+    run_ring_rope(3, 1, 4000, 1, [2, 2], seed=79)
 
 
 def test_ring_rope_rejects_grid_mismatch():
