@@ -9,7 +9,7 @@ CPU fallback).
 
 import importlib
 
-_SUBMODULES = ("rkv", "synth", "build")
+_SUBMODULES = ("rkv", "synth", "build", "shard")
 __all__ = list(_SUBMODULES)
 
 
