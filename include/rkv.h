@@ -120,7 +120,9 @@ rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H, int32_t D,
  * "Three problems for generic compilers").
  *
  *   q, k, v       device bf16 [Lq][H][D], [Lk][H][D], [Lk][H][D]
- *   o             device bf16 [Lq][H][D]; must not overlap q, k or v
+ *   o             device bf16 [Lq][H][D]; may share no byte with any q, k, v
+ *                 or other o of the launch (row-strided views with disjoint
+ *                 heads of one tensor, e.g. head slices, are fine)
  *   *_stride      elements between consecutive rows (>= H*D, 16-B aligned rows)
  *   Lq, Lk        >= 1 each
  *   q_t0, k_t0    time index of the first query / key frame (used for RoPE)

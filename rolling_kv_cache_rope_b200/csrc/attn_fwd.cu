@@ -1091,8 +1091,6 @@ static rkv_status validate_seq(const rkv_attn_seq& s, int i, int32_t H) {
   return RKV_OK;
 }
 
-static uint64_t span_bytes(int64_t L, int64_t stride, int32_t H) { return uint64_t((L - 1) * stride + int64_t(H) * kHD) * 2; }
-
 extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
                                       float softmax_scale, const rkv_rope3d* rope, void* workspace,
                                       size_t workspace_bytes, void* stream) {
@@ -1110,14 +1108,17 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
     st = validate_seq(seqs[i], i, H);
     if (st != RKV_OK) return st;
   }
+  // outputs may not share a byte with any input or other output; row-strided
+  // views of one tensor with disjoint heads (a launch over head slices) pass
+  const int64_t row_bytes = int64_t(H) * kHD * 2;
   for (int i = 0; i < n_seqs; ++i) {
-    const uint64_t ob = span_bytes(seqs[i].Lq, seqs[i].o_stride, H);
+    const rkv_attn_seq& s = seqs[i];
     for (int j = 0; j < n_seqs; ++j) {
       const rkv_attn_seq& t = seqs[j];
-      if (overlaps(seqs[i].o, ob, t.q, span_bytes(t.Lq, t.q_stride, H)) ||
-          overlaps(seqs[i].o, ob, t.k, span_bytes(t.Lk, t.k_stride, H)) ||
-          overlaps(seqs[i].o, ob, t.v, span_bytes(t.Lk, t.v_stride, H)) ||
-          (i != j && overlaps(seqs[i].o, ob, t.o, span_bytes(t.Lq, t.o_stride, H))))
+      if (rows_overlap(s.o, s.Lq, s.o_stride * 2, row_bytes, t.q, t.Lq, t.q_stride * 2, row_bytes) ||
+          rows_overlap(s.o, s.Lq, s.o_stride * 2, row_bytes, t.k, t.Lk, t.k_stride * 2, row_bytes) ||
+          rows_overlap(s.o, s.Lq, s.o_stride * 2, row_bytes, t.v, t.Lk, t.v_stride * 2, row_bytes) ||
+          (i != j && rows_overlap(s.o, s.Lq, s.o_stride * 2, row_bytes, t.o, t.Lq, t.o_stride * 2, row_bytes)))
         return fail(RKV_ERR_INVALID_ARG, "seq %d: output overlaps an input or another output", i);
     }
   }

@@ -47,6 +47,28 @@ inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return na && nb && x < y + nb && y < x + na;
 }
 
+// Do two row-strided byte ranges share a byte?  Range X holds rows
+// [x + i * stride, x + i * stride + width), i < rows.  With equal strides the
+// answer is exact: rows i of A and j of B meet iff, for k = i - j,
+// d - width_a < k * stride < d + width_b with d = b - a; so it is enough to
+// test the smallest k above (d - width_a) / stride that is a possible i - j.
+// Head-sliced views of one tensor (same stride, disjoint columns) therefore
+// do not overlap.  Different strides fall back to the byte spans.
+inline bool rows_overlap(const void* a, int64_t rows_a, int64_t stride_a, int64_t width_a, const void* b,
+                         int64_t rows_b, int64_t stride_b, int64_t width_b) {
+  if (rows_a < 1 || rows_b < 1 || width_a < 1 || width_b < 1) return false;
+  const uint64_t span_a = uint64_t((rows_a - 1) * stride_a + width_a);
+  const uint64_t span_b = uint64_t((rows_b - 1) * stride_b + width_b);
+  if (!overlaps(a, span_a, b, span_b)) return false;
+  if (stride_a != stride_b || width_a > stride_a || width_b > stride_b) return true;
+  const int64_t S = stride_a;
+  const int64_t d = int64_t(reinterpret_cast<uintptr_t>(b)) - int64_t(reinterpret_cast<uintptr_t>(a));
+  const int64_t lo = d - width_a;                           // k * S must exceed lo
+  int64_t k = (lo >= 0 ? lo / S : -((-lo + S - 1) / S)) + 1;  // floor(lo / S) + 1
+  if (k < -(rows_b - 1)) k = -(rows_b - 1);
+  return k <= rows_a - 1 && k * S < d + width_b;
+}
+
 // ---- unsigned division by a run-time constant -----------------------------
 // floor(n / d) = (umulhi(n, m) + n) >> s for every n < 2^31, with
 // s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1 (Granlund and

@@ -13,7 +13,8 @@ rows of frame f and head h's whole K and V.  Rank r takes a contiguous run
 of units in head-major order, the runs differing in length by at most one
 unit, so there is no padding and no cut inside a frame; when world divides
 H every rank holds whole heads.  A rank's run is a few segments (h, f0, f1)
-that become single-head sequences of ONE attention launch: the query view
+that become single-head sequences of ONE attention launch (one view of
+several heads when the rank holds whole heads): the query view
 starts at frame f0, so its time index is q_t0 + f0 and its mask offset
 q_frame_offset + f0 (the (h, w) position of a row depends only on the row
 within its frame).  The ring of each layer shards by heads the same way (a
@@ -81,15 +82,30 @@ def _query_frames(seq, F):
 
 
 def shard_seqs(seqs, F, rank, world, kv_head0=0):
-    """The single-head AttnSeqs of ``rank``'s units of every sequence (views of
-    the callers' tensors; no copies).  Q and O hold every head; K and V hold
-    heads from ``kv_head0`` on (a rank's own ring holds only the heads its
-    units touch: kv_head0 = that run's first head)."""
+    """The AttnSeqs of ``rank``'s units of every sequence (views of the
+    callers' tensors; no copies): one view of its heads per sequence when
+    every rank holds whole heads, else one single-head view per segment (one
+    launch takes at most 16).  Q and O hold every head; K and V hold heads
+    from ``kv_head0`` on (a rank's own ring holds only the heads its units
+    touch: kv_head0 = that run's first head)."""
     from .rkv import AttnSeq
+    runs = [unit_runs(seq.q.shape[1], _query_frames(seq, F), world)[rank] for seq in seqs]
+    whole = [all((f0, f1) == (0, r.q_frames) for _, f0, f1 in r.segments()) for r in runs]
+    if all(whole) and len({r.heads()[1] - r.heads()[0] for r in runs}) == 1:
+        # whole heads everywhere (world divides H): one multi-head view per sequence
+        out = []
+        for seq, r in zip(seqs, runs):
+            h0, h1 = r.heads()
+            if h0 - kv_head0 < 0 or h1 - kv_head0 > seq.k.shape[1]:
+                raise ValueError(f"heads [{h0}, {h1}) are not among the K/V heads starting at {kv_head0}")
+            hs, kv = slice(h0, h1), slice(h0 - kv_head0, h1 - kv_head0)
+            s = AttnSeq(seq.q[:, hs], seq.k[:, kv], seq.v[:, kv], seq.o[:, hs], q_t0=seq.q_t0, k_t0=seq.k_t0,
+                        block_frames=seq.block_frames, q_frame_offset=seq.q_frame_offset)
+            s.flags = seq.flags
+            out.append(s)
+        return out
     out = []
-    for seq in seqs:
-        H = seq.q.shape[1]
-        run = unit_runs(H, _query_frames(seq, F), world)[rank]
+    for seq, run in zip(seqs, runs):
         for h, f0, f1 in run.segments():
             rows, hs, kv = slice(f0 * F, f1 * F), slice(h, h + 1), slice(h - kv_head0, h - kv_head0 + 1)
             if not 0 <= h - kv_head0 < seq.k.shape[1]:

@@ -234,6 +234,29 @@ def test_attn_rejects(rkv, kw, frag):
     assert frag in rkv.rkv_last_error_string()
 
 
+def test_attn_outputs_may_be_head_slices_of_one_tensor(rkv):
+    # four single-head sequences whose Q/O are heads 0..3 of [72, 4, 128]
+    # tensors (row stride 4 heads): the strided outputs share no byte, so the
+    # host checks pass (the launch itself then fails without a GPU)
+    lib = rkv.lib()
+    r = rope(rkv)
+    q0, o0, k0 = 0x1000000, 0x2000000, 0x3000000
+    def head_seq(h, o_head=None):
+        return seq(rkv, q=q0 + h * 256, o=o0 + (h if o_head is None else o_head) * 256, k=k0 + h * 256,
+                   v=k0 + 0x800000 + h * 256, q_stride=512, k_stride=512, v_stride=512, o_stride=512)
+    arr = (rkv.rkv_attn_seq * 4)(*[head_seq(h) for h in range(4)])
+    st = lib.attn_fwd_varlen(arr, 4, 1, 128, 0.088, ctypes.byref(r), fake(0x700000), 256, None)
+    assert "overlaps" not in rkv.rkv_last_error_string() and st != rkv.RKV_ERR_INVALID_ARG, \
+        rkv.rkv_last_error_string()
+    # two sequences writing the same head, or an output on another's input
+    for bad in ([head_seq(0), head_seq(1, o_head=0)],
+                [head_seq(0), seq(rkv, q=o0, o=o0 + 2 * 256, k=k0, v=k0 + 0x800000, q_stride=512,
+                                  k_stride=512, v_stride=512, o_stride=512)]):
+        arr = (rkv.rkv_attn_seq * 2)(*bad)
+        st = lib.attn_fwd_varlen(arr, 2, 1, 128, 0.088, ctypes.byref(r), fake(0x700000), 256, None)
+        assert st == rkv.RKV_ERR_INVALID_ARG and "overlaps" in rkv.rkv_last_error_string()
+
+
 def test_attn_rejects_launch_level_arguments(rkv):
     lib = rkv.lib()
     arr = (rkv.rkv_attn_seq * 1)(seq(rkv))

@@ -65,6 +65,27 @@ def test_more_ranks_than_units_is_an_error():
         unit_runs(0, 3, 1)
 
 
+def test_whole_head_runs_become_one_view_per_sequence():
+    import torch
+    from rolling_kv_cache_rope_b200.rkv import AttnSeq
+    from rolling_kv_cache_rope_b200.shard import shard_seqs
+    q = torch.zeros((3 * 6, 4, 128), dtype=torch.bfloat16)
+    k = torch.zeros((5 * 6, 4, 128), dtype=torch.bfloat16)
+    o = torch.zeros_like(q)
+    seq = AttnSeq(q, k, k, o, q_t0=2, k_t0=0, block_frames=1, q_frame_offset=2)
+    for rank in range(2):
+        (s,) = shard_seqs([seq], 6, rank, 2)
+        assert s.q.shape == (18, 2, 128) and s.k.shape == (30, 2, 128)
+        assert s.q.data_ptr() == q.data_ptr() + rank * 2 * 128 * 2
+        assert s.o.data_ptr() == o.data_ptr() + rank * 2 * 128 * 2
+        assert (s.q_t0, s.q_frame_offset, s.block_frames, s.flags) == (2, 2, 1, seq.flags)
+    # K/V holding only rank 1's heads
+    (s,) = shard_seqs([AttnSeq(q, k[:, 2:], k[:, 2:], o)], 6, 1, 2, kv_head0=2)
+    assert s.k.data_ptr() == k.data_ptr() + 2 * 128 * 2
+    with pytest.raises(ValueError):
+        shard_seqs([AttnSeq(q, k[:, 2:], k[:, 2:], o)], 6, 0, 2, kv_head0=2)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -100,6 +121,8 @@ def _rank_main(rank, world, port, results):
         whole = AttnSeq(q, k, v, o, q_t0=Q_T0, k_t0=0, block_frames=BLOCK, q_frame_offset=Q_T0)
         pieces = shard_seqs([whole], F, rank, world)
         segs = unit_runs(H, QF, world)[rank].segments()
+        if world == H:   # whole heads: one view of the rank's head
+            assert len(pieces) == 1 and pieces[0].q.shape == (QF * F, 1, D)
         assert len(pieces) == len(segs)
         for s, (h, f0, f1) in zip(pieces, segs):
             assert s.q.shape == (s.o.shape[0], 1, D) and s.k.shape == (KF * F, 1, D)
@@ -117,7 +140,7 @@ def _rank_main(rank, world, port, results):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 5])
 def test_sharded_units_reassemble_to_the_whole_sequence(world):
     from oracle import bf16_bits_to_f64, bf16_ulp_distance, f64_to_bf16_bits, fused_attention_ref
     from rolling_kv_cache_rope_b200.synth import bf16_normal_bits
