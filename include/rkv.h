@@ -11,7 +11,9 @@
  *                        cache-update pass) in one launch, optional
  *                        frame-block-causal mask
  *   kvcache_ring_update  insert whole frames into a per-layer ring cache,
- *                        evicting the oldest frames
+ *                        evicting the oldest frames (optionally keeping a
+ *                        pinned prefix of first frames);
+ *                        kvcache_ring_update_rope rotates K on the way in
  *
  * Conventions shared by every call
  * --------------------------------
@@ -26,8 +28,9 @@
  *  - Every call returns an rkv_status.  Invalid arguments are rejected on the
  *    host BEFORE anything is launched; nothing traps or asserts on the device.
  *    rkv_last_error_string() describes the last failure of the calling thread.
- *  - Functions keep no global state between calls (the ring state lives in the
- *    caller's rkv_ring).
+ *  - Functions keep no state between calls (the ring state lives in the
+ *    caller's rkv_ring) except two fixed device words per GPU: the status of
+ *    attn_fwd_varlen_noalloc and the ring inserts' timeout flag.
  */
 #ifndef RKV_H
 #define RKV_H
