@@ -346,15 +346,13 @@ static rkv_status launch_rope_shape(RopeArgs& a, int64_t L, int32_t H, int32_t t
   a.rows_per_cta = uint32_t(rpc);
   const int64_t grid = (L + rpc - 1) / rpc;
   const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing, kHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kRopeMaxEntries * int(sizeof(TabEntry)));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
-    attr_set = true;
-  }
+  // set on every launch: the attribute belongs to the current device, and a
+  // process may launch on several
+  cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing, kHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kRopeMaxEntries * int(sizeof(TabEntry)));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
   rope3d_kernel<kRing, kHalf><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
   return RKV_OK;
 }
