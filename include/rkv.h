@@ -187,6 +187,32 @@ rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, 
                            size_t workspace_bytes, void* stream);
 
 /*
+ * rkv_attn_mask_rows -- the mask and key-tile plan attn_fwd_varlen would use,
+ * evaluated on the host by the same functions the kernel compiles (a debug
+ * and test aid; needs no GPU).  The frame-block-causal mask ("Amazon and
+ * Reactor tune Trainium for real-time video generation", section "Three
+ * problems for generic compilers", the two passes of different lengths) makes
+ * every query row see a prefix of the keys, so a row's mask is one number.
+ *
+ *   seqs, n_seqs, H, rope   as for attn_fwd_varlen; only Lq, Lk,
+ *                  q_frame_offset, block_frames and the frame grid are read
+ *                  (tensor pointers and strides may be anything)
+ *   row_limit      host int64 [sum of Lq]: for sequence i (in the order given)
+ *                  and its query row r, entry Lq_0 + ... + Lq_{i-1} + r is the
+ *                  number of leading keys row r attends to; keys at or past it
+ *                  are masked
+ *   unit_tiles     optional host int32 [4 * n_units]: per work unit in launch
+ *                  order, (sequence index in the order given, head, 512-row
+ *                  query block, key tiles of 128 keys the unit processes)
+ *   n_units        optional out: number of work units, sum of H * ceil(Lq / 512)
+ * Errors: RKV_ERR_INVALID_ARG (as attn_fwd_varlen for n_seqs, H, rope,
+ * lengths, mask fields; row_limit NULL), RKV_ERR_UNSUPPORTED (n_seqs > 16).
+ */
+rkv_status rkv_attn_mask_rows(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, const rkv_rope3d* rope,
+                              int64_t* row_limit, int32_t* unit_tiles, int64_t* n_units);
+
+/*
+ * rkv_attn_status -- synchronise/*
  * rkv_attn_status -- synchronise `stream` and return the device status word
  * an earlier attn_fwd_varlen left in `workspace` (RKV_OK or RKV_ERR_TIMEOUT),
  * then clear it.

@@ -202,7 +202,11 @@ struct Unit {
   int part;       // -1: whole unit; else index of the item's partial-result slot
 };
 
-__device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p, int row) {
+// Keys [0, limit) of the sequence are visible to query row `row`: the whole
+// context without a mask, else every key frame up to the end of the query
+// frame's block.  Host and device share this code (the host evaluates it for
+// the tail split and for rkv_attn_mask_rows).
+__host__ __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p, int row) {
   if (s.block_frames <= 0) return s.Lk;
   const int64_t qf = int64_t(s.q_frame_offset) + row / int64_t(p.F);
   const int64_t blk = qf / s.block_frames;
@@ -214,7 +218,7 @@ __device__ __forceinline__ int64_t row_kv_limit(const SeqDev& s, const Params& p
 // sequence (all query blocks of head 0, then head 1, ...), so the clusters in
 // flight at any time share the K/V tiles of one or two heads in L2.  Masked
 // sequences list their query blocks from the most to the least visible keys.
-__device__ __forceinline__ Unit decode_unit(const Params& p, int item) {
+__host__ __device__ __forceinline__ Unit decode_unit(const Params& p, int item) {
   Unit r;
   int u = item;
   r.part = -1;
@@ -1091,6 +1095,32 @@ static rkv_status validate_seq(const rkv_attn_seq& s, int i, int32_t H) {
   return RKV_OK;
 }
 
+// Launch order of the sequences (longest context first: the cheapest units
+// come last, which helps the static schedule) and each one's fields that
+// number and size its work units; returns the number of units.  Fills p.F,
+// p.n_seqs, p.H and p.n_whole (= all units, before any tail split).
+static int64_t plan_units(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int64_t F, Params& p,
+                          int* order) {
+  for (int i = 0; i < n_seqs; ++i) order[i] = i;
+  for (int i = 1; i < n_seqs; ++i)
+    for (int j = i; j > 0 && seqs[order[j]].Lk > seqs[order[j - 1]].Lk; --j) std::swap(order[j], order[j - 1]);
+  int64_t units = 0;
+  for (int oi = 0; oi < n_seqs; ++oi) {
+    const rkv_attn_seq& s = seqs[order[oi]];
+    SeqDev& d = p.seq[oi];
+    d.Lq = s.Lq; d.Lk = s.Lk; d.q_t0 = s.q_t0; d.k_t0 = s.k_t0;
+    d.q_frame_offset = s.q_frame_offset; d.block_frames = s.block_frames; d.flags = s.flags;
+    d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;   // 512-row blocks, one per CTA pair
+    d.unit_begin = int32_t(units);
+    units += int64_t(d.n_qblocks) * H;
+  }
+  p.F = uint32_t(F);
+  p.n_seqs = n_seqs;
+  p.H = H;
+  p.n_whole = int32_t(units < INT32_MAX ? units : INT32_MAX);
+  return units;
+}
+
 extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
                                       float softmax_scale, const rkv_rope3d* rope, void* workspace,
                                       size_t workspace_bytes, void* stream) {
@@ -1126,14 +1156,10 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   Params p;
   memset(&p, 0, sizeof(p));
   const int64_t F = int64_t(rope->grid_h) * rope->grid_w;
-  // order: longest context first (cheapest-last helps the static schedule)
   int order[RKV_MAX_SEQS];
-  for (int i = 0; i < n_seqs; ++i) order[i] = i;
-  for (int i = 1; i < n_seqs; ++i)
-    for (int j = i; j > 0 && seqs[order[j]].Lk > seqs[order[j - 1]].Lk; --j) std::swap(order[j], order[j - 1]);
+  const int64_t units = plan_units(seqs, n_seqs, H, F, p, order);
 
   int64_t t_lo = INT64_MAX, t_hi = INT64_MIN;
-  int64_t units = 0;
   for (int oi = 0; oi < n_seqs; ++oi) {
     const rkv_attn_seq& s = seqs[order[oi]];
     SeqDev& d = p.seq[oi];
@@ -1142,11 +1168,6 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
     if ((st = make_map(&d.tv, s.v, s.Lk, H, s.v_stride, kBN)) != RKV_OK) return st;
     d.o = static_cast<uint8_t*>(s.o);
     d.o_stride_bytes = s.o_stride * 2;
-    d.Lq = s.Lq; d.Lk = s.Lk; d.q_t0 = s.q_t0; d.k_t0 = s.k_t0;
-    d.q_frame_offset = s.q_frame_offset; d.block_frames = s.block_frames; d.flags = s.flags;
-    d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;   // 512-row blocks, one per CTA pair
-    d.unit_begin = int32_t(units);
-    units += int64_t(d.n_qblocks) * H;
     if (s.flags & RKV_ROPE_Q) {
       t_lo = std::min<int64_t>(t_lo, s.q_t0);
       t_hi = std::max<int64_t>(t_hi, int64_t(s.q_t0) + (s.Lq - 1) / F);
@@ -1234,11 +1255,7 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
     const int qb = d.block_frames > 0 ? (d.n_qblocks - 1 - ord) : ord;
     int64_t last = int64_t(qb + 1) * kUnitRows - 1;
     if (last > d.Lq - 1) last = d.Lq - 1;
-    int64_t kv = d.Lk;
-    if (d.block_frames > 0) {
-      const int64_t qf = int64_t(d.q_frame_offset) + last / F;
-      kv = std::min<int64_t>((qf / d.block_frames + 1) * d.block_frames * F, d.Lk);
-    }
+    const int64_t kv = row_kv_limit(d, p, int(last));
     if ((kv + kBN - 1) / kBN < 2) { n_split = 0; break; }
     ca.unit[k].o = d.o;
     ca.unit[k].o_stride_bytes = d.o_stride_bytes;
@@ -1268,6 +1285,48 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attn_combine_kernel launch");
   }
+  return RKV_OK;
+}
+
+extern "C" rkv_status rkv_attn_mask_rows(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H,
+                                         const rkv_rope3d* rope, int64_t* row_limit, int32_t* unit_tiles,
+                                         int64_t* n_units) {
+  clear_error();
+  if (!seqs || n_seqs < 1) return fail(RKV_ERR_INVALID_ARG, "need at least one sequence");
+  if (n_seqs > RKV_MAX_SEQS) return fail(RKV_ERR_UNSUPPORTED, "at most %d sequences per launch", RKV_MAX_SEQS);
+  if (H < 1) return fail(RKV_ERR_INVALID_ARG, "H must be >= 1");
+  rkv_status st = check_rope(rope, kHD);
+  if (st != RKV_OK) return st;
+  if (!row_limit) return fail(RKV_ERR_INVALID_ARG, "row_limit is NULL");
+  for (int i = 0; i < n_seqs; ++i) {
+    const rkv_attn_seq& s = seqs[i];
+    if (s.Lq < 1 || s.Lk < 1) return fail(RKV_ERR_INVALID_ARG, "seq %d: Lq and Lk must be >= 1", i);
+    if (s.block_frames < 0) return fail(RKV_ERR_INVALID_ARG, "seq %d: block_frames < 0", i);
+    if (s.block_frames > 0 && s.q_frame_offset < 0)
+      return fail(RKV_ERR_INVALID_ARG, "seq %d: q_frame_offset must be >= 0 with a mask", i);
+  }
+  Params p;
+  memset(&p, 0, sizeof(p));
+  int order[RKV_MAX_SEQS], where[RKV_MAX_SEQS];
+  const int64_t units = plan_units(seqs, n_seqs, H, int64_t(rope->grid_h) * rope->grid_w, p, order);
+  if (units >= (int64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "too many work units");
+  for (int oi = 0; oi < n_seqs; ++oi) where[order[oi]] = oi;
+  int64_t off = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const SeqDev& d = p.seq[where[i]];
+    for (int r = 0; r < d.Lq; ++r) row_limit[off + r] = row_kv_limit(d, p, r);
+    off += d.Lq;
+  }
+  if (unit_tiles) {
+    for (int64_t u = 0; u < units; ++u) {
+      const Unit un = decode_unit(p, int(u));
+      unit_tiles[4 * u + 0] = order[un.si];
+      unit_tiles[4 * u + 1] = un.head;
+      unit_tiles[4 * u + 2] = un.qb;
+      unit_tiles[4 * u + 3] = un.nkt;
+    }
+  }
+  if (n_units) *n_units = units;
   return RKV_OK;
 }
 

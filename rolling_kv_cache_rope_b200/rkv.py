@@ -62,6 +62,9 @@ _lib.attn_fwd_varlen.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int3
                                  _c.POINTER(rkv_rope3d), _c.c_void_p, _c.c_size_t, _c.c_void_p]
 _lib.rkv_attn_status.restype = _c.c_int
 _lib.rkv_attn_status.argtypes = [_c.c_void_p, _c.c_void_p]
+_lib.rkv_attn_mask_rows.restype = _c.c_int
+_lib.rkv_attn_mask_rows.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int32, _c.POINTER(rkv_rope3d),
+                                    _c.POINTER(_c.c_int64), _c.POINTER(_c.c_int32), _c.POINTER(_c.c_int64)]
 _lib.kvcache_ring_update.restype = _c.c_int
 _lib.kvcache_ring_update.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
                                      _c.POINTER(_c.c_int32), _c.c_void_p]
@@ -188,6 +191,42 @@ def attn_fwd_varlen(seqs, rope, softmax_scale=None, workspace=None, stream=None)
 def rkv_attn_status(workspace, stream=None):
     """Synchronise and raise RkvError if the last launch on ``workspace`` timed out."""
     _check(_lib.rkv_attn_status(workspace.data_ptr(), _stream(stream)))
+
+
+def attn_mask_rows(seqs, H, rope):
+    """The mask and key-tile plan attn_fwd_varlen uses for ``seqs``, evaluated
+    on the host by the kernel's own code (no GPU needed).  ``seqs``: AttnSeq
+    objects or dicts with Lq, Lk and optional q_frame_offset, block_frames.
+    Returns (limits, units): limits[i][r] = keys visible to query row r of
+    sequence i (a prefix); units = int32 [n_units, 4] rows of (sequence,
+    head, 512-row query block, 128-key tiles processed), in launch order."""
+    import numpy as np
+    descs = []
+    for s in seqs:
+        if isinstance(s, dict):
+            descs.append(rkv_attn_seq(Lq=int(s["Lq"]), Lk=int(s["Lk"]), q_frame_offset=int(s.get("q_frame_offset", 0)),
+                                      block_frames=int(s.get("block_frames", 0))))
+        else:
+            descs.append(rkv_attn_seq(Lq=int(s.q.shape[0]), Lk=int(s.k.shape[0]), q_frame_offset=s.q_frame_offset,
+                                      block_frames=s.block_frames))
+    if not descs:
+        raise ValueError("need at least one sequence")
+    arr = (rkv_attn_seq * len(descs))(*descs)
+    lq = [d.Lq for d in descs]
+    limits = np.zeros(max(1, sum(lq)), dtype=np.int64)
+    n_units = sum(int(H) * ((x + 511) // 512) for x in lq)
+    units = np.zeros((max(1, n_units), 4), dtype=np.int32)
+    got = ctypes.c_int64(0)
+    _check(_lib.rkv_attn_mask_rows(arr, len(descs), int(H), ctypes.byref(rope),
+                                   limits.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                   units.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), ctypes.byref(got)))
+    if got.value != n_units:
+        raise RuntimeError(f"unit count {got.value} != {n_units}")
+    out, at = [], 0
+    for x in lq:
+        out.append(limits[at:at + x].copy())
+        at += x
+    return out, units[:n_units]
 
 
 def rkv_ring_status(stream=None):
