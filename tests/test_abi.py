@@ -257,6 +257,50 @@ def test_attn_outputs_may_be_head_slices_of_one_tensor(rkv):
         assert st == rkv.RKV_ERR_INVALID_ARG and "overlaps" in rkv.rkv_last_error_string()
 
 
+def _views_share_a_byte(a, la, sa, b, lb, sb, width):
+    return any(a + i * sa < b + j * sb + width and b + j * sb < a + i * sa + width
+               for i in range(la) for j in range(lb))
+
+
+def test_attn_output_overlap_check_is_exact(rkv):
+    # random pairs of row-strided single-head views (row = 256 bytes): with
+    # equal row strides the host check flags an output exactly when it shares
+    # a byte with another sequence's output or input (brute force over the
+    # rows); with different strides it flags overlapping byte spans
+    from hypothesis import given, settings, strategies as st
+    lib = rkv.lib()
+    r = rope(rkv)
+    base = 0x10000000
+
+    @settings(max_examples=300, deadline=None)
+    @given(st.integers(1, 5), st.integers(1, 5), st.sampled_from([128, 136, 256, 384, 512]),
+           st.sampled_from([128, 256, 384, 512]), st.integers(0, 40), st.booleans())
+    def check(la, lb, sa, sb, off16, against_output):
+        a_o = base
+        b_t = base + off16 * 16
+        far = 0x40000000
+        sa_ = sa
+        sb_ = sb
+        A = seq(rkv, q=far, k=far + 0x1000000, v=far + 0x2000000, o=a_o, q_stride=sa_, k_stride=128, v_stride=128,
+                o_stride=sa_, Lq=la, Lk=8, q_t0=0, q_frame_offset=0, flags=0)
+        if against_output:
+            B = seq(rkv, q=far + 0x3000000, k=far + 0x4000000, v=far + 0x5000000, o=b_t, q_stride=sb_,
+                    k_stride=128, v_stride=128, o_stride=sb_, Lq=lb, Lk=8, q_t0=0, q_frame_offset=0, flags=0)
+        else:
+            B = seq(rkv, q=b_t, k=far + 0x4000000, v=far + 0x5000000, o=far + 0x6000000, q_stride=sb_,
+                    k_stride=128, v_stride=128, o_stride=sb_, Lq=lb, Lk=8, q_t0=0, q_frame_offset=0, flags=0)
+        arr = (rkv.rkv_attn_seq * 2)(A, B)
+        lib.attn_fwd_varlen(arr, 2, 1, 128, 0.088, ctypes.byref(r), fake(0x700000), 256, None)
+        flagged = "overlaps" in rkv.rkv_last_error_string()
+        if sa == sb:
+            want = _views_share_a_byte(a_o, la, sa_ * 2, b_t, lb, sb_ * 2, 256)
+        else:   # different row strides: the byte spans decide (conservative)
+            want = a_o < b_t + (lb - 1) * sb_ * 2 + 256 and b_t < a_o + (la - 1) * sa_ * 2 + 256
+        assert flagged == want, (la, lb, sa, sb, off16, against_output)
+
+    check()
+
+
 def test_attn_rejects_launch_level_arguments(rkv):
     lib = rkv.lib()
     arr = (rkv.rkv_attn_seq * 1)(seq(rkv))
