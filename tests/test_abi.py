@@ -106,6 +106,34 @@ def test_ring_slot_pinned_matches_oracle(rkv):
     assert lib.rkv_ring_slot(ctypes.byref(bad), 0) == -1
 
 
+def test_ring_insert_capacity_matches_oracle(rkv):
+    # over random reachable states of pinned rings, an insert is refused on
+    # the host exactly when the oracle ring says it carries too many frames
+    # (an accepted one then fails at the launch here: no GPU) and the state
+    # is left unchanged either way
+    from hypothesis import given, settings, strategies as st
+    from oracle import RingRef
+    lib = rkv.lib()
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.integers(1, 9), st.data())
+    def check(W, data):
+        P = data.draw(st.integers(0, W - 1))
+        ref = RingRef(W, P)
+        for n in data.draw(st.lists(st.integers(0, W), max_size=6)):
+            if n <= ref.capacity_for_insert():
+                ref.insert([None] * n)
+        n = data.draw(st.integers(0, W + 1))
+        r = ring(rkv, slots=W, head=ref.head, count=ref.count, pinned=P)
+        st_ = lib.kvcache_ring_update(ctypes.byref(r), fake(0x40000000), fake(0x50000000), 2 * 128, n, None, None)
+        refused = st_ == rkv.RKV_ERR_INVALID_ARG and "n_frames" in rkv.rkv_last_error_string()
+        assert refused == (n > ref.capacity_for_insert()), (W, P, ref.head, ref.count, n, st_)
+        if n > 0:
+            assert (r.head, r.count) == (ref.head, ref.count)
+
+    check()
+
+
 def test_ring_update_rejects_bad_sources(rkv):
     lib = rkv.lib()
     r = ring(rkv)

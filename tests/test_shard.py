@@ -42,6 +42,22 @@ def test_runs_partition_the_units(H, q_frames, world):
     assert max(sizes) - min(sizes) <= 1 and sum(sizes) == H * q_frames
 
 
+def test_runs_partition_random_shapes():
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(st.integers(1, 40), st.integers(1, 30), st.data())
+    def check(H, q_frames, data):
+        world = data.draw(st.integers(1, min(64, H * q_frames)))
+        test_runs_partition_the_units(H, q_frames, world)
+        # a rank touches at most ceil(units / q_frames) + 1 heads
+        for r in unit_runs(H, q_frames, world):
+            h0, h1 = r.heads()
+            assert h1 - h0 <= -(-r.units // q_frames) + 1
+
+    check()
+
+
 def test_whole_heads_when_world_divides_heads():
     for world in (1, 2, 3, 4, 6, 12):
         for r in unit_runs(12, 15, world):
