@@ -17,8 +17,11 @@ that become single-head sequences of ONE attention launch (one view of
 several heads when the rank holds whole heads): the query view
 starts at frame f0, so its time index is q_t0 + f0 and its mask offset
 q_frame_offset + f0 (the (h, w) position of a row depends only on the row
-within its frame).  The ring of each layer shards by heads the same way (a
-rank keeps the heads its units touch).  Nothing is exchanged inside
+within its frame).  The ring of each layer shards by heads the same way: a
+rank keeps the heads [h0, h1) = unit_runs(...)[rank].heads() its units touch,
+in a KVRing of h1 - h0 heads fed with the head slices k_new[:, h0:h1] and
+v_new[:, h0:h1] (strided views the ring insert accepts), and passes
+kv_head0 = h0 when it attends over that ring.  Nothing is exchanged inside
 attention; the one collective is the all-gather of the outputs for a
 consumer that needs every head of every row (the output projection, outside
 this library).
