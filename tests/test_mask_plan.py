@@ -72,6 +72,31 @@ def test_ragged_tails_and_several_sequences(rkv):
     check_dense(rkv, specs, 3, 4, 6)
 
 
+def test_random_shapes(rkv):
+    # random grids, lengths (ragged tails included), mask blocks and query
+    # offsets, several sequences per launch
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=120, deadline=None)
+    @given(st.integers(1, 4), st.integers(1, 5), st.integers(1, 3), st.data())
+    def check(gh, gw, H, data):
+        F = gh * gw
+        specs = []
+        for _ in range(data.draw(st.integers(1, 4))):
+            kf = data.draw(st.integers(1, 40))
+            Lk = kf * F - data.draw(st.integers(0, F - 1))
+            block = data.draw(st.sampled_from([0, 1, 2, 3, 5]))
+            if block:
+                qf = data.draw(st.integers(1, kf))
+                specs.append(dict(Lq=qf * F, Lk=Lk, q_frame_offset=data.draw(st.integers(0, kf - qf)),
+                                  block_frames=block))
+            else:
+                specs.append(dict(Lq=data.draw(st.integers(1, 700)), Lk=Lk))
+        check_dense(rkv, specs, H, gh, gw)
+
+    check()
+
+
 def test_full_size_two_pass_launch(rkv):
     F = TWO_PASS_DENOISE.frame_tokens
     specs = []
