@@ -361,7 +361,11 @@ int32_t rkv_ring_slot(const rkv_ring* ring, int32_t logical_frame);
 /* Text of the last error returned on the calling thread ("" if none). */
 const char* rkv_last_error_string(void);
 
-/* Library version, major*10000 + minor*100 + patch. */
+/* Library version, major*10000 + minor*100 + patch.  A caller compiled
+ * against this header can compare it with RKV_VERSION: the structs above
+ * changed layout between minor versions (rkv_ring gained `pinned`,
+ * rkv_rope3d its per-axis bases and layout in 0.2). */
+#define RKV_VERSION 200
 int32_t rkv_version(void);
 
 #ifdef __cplusplus

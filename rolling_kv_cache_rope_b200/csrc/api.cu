@@ -33,4 +33,4 @@ rkv_status cuda_fail(cudaError_t e, const char* what) {
 
 extern "C" const char* rkv_last_error_string(void) { return rkv::g_last_error; }
 
-extern "C" int32_t rkv_version(void) { return 100; /* 0.1.0 */ }
+extern "C" int32_t rkv_version(void) { return RKV_VERSION; }
