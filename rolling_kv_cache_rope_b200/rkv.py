@@ -242,6 +242,8 @@ class KVRing:
 
     def __init__(self, slots, tokens_per_frame, H, D=128, device="cuda", k=None, v=None, pinned=0):
         import torch
+        if not 0 <= pinned < slots:
+            raise ValueError(f"pinned ({pinned}) must be in [0, slots={slots})")
         shape = (slots, tokens_per_frame, H, D)
         self.k = torch.empty(shape, dtype=torch.bfloat16, device=device) if k is None else k
         self.v = torch.empty(shape, dtype=torch.bfloat16, device=device) if v is None else v
