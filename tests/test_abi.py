@@ -346,6 +346,13 @@ def test_attn_rejects_launch_level_arguments(rkv):
     assert lib.attn_fwd_varlen_workspace_size(arr, 1, 2, 128) >= 4
 
 
+def test_kvring_refuses_pinned_prefix_without_rolling_slot(rkv):
+    with pytest.raises(ValueError):
+        rkv.KVRing(3, 24, 2, pinned=3, device="cpu")
+    r = rkv.KVRing(3, 24, 2, pinned=2, device="cpu")
+    assert (r.head, r.count, r.pinned) == (2, 0, 2)
+
+
 def test_python_binding_refuses_non_bf16(rkv):
     import torch
     x = torch.zeros(4, 2, 128, dtype=torch.float32)
