@@ -47,7 +47,8 @@ typedef enum {
   RKV_ERR_INVALID_ARG = 1, /* rejected on the host, nothing launched           */
   RKV_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels handle  */
   RKV_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed                */
-  RKV_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see below)   */
+  RKV_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (see below)   */
+  RKV_ERR_DEVICE_CHECK = 5 /* a debug launch's device-side index check failed  */
 } rkv_status;
 
 /*
@@ -212,12 +213,70 @@ rkv_status rkv_attn_mask_rows(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t 
                               int64_t* row_limit, int32_t* unit_tiles, int64_t* n_units);
 
 /*
- * rkv_attn_status -- synchronise/*
  * rkv_attn_status -- synchronise `stream` and return the device status word
  * an earlier attn_fwd_varlen left in `workspace` (RKV_OK or RKV_ERR_TIMEOUT),
  * then clear it.
  */
 rkv_status rkv_attn_status(void* workspace, void* stream);
+
+/*
+ * attn_fwd_varlen_debug -- attn_fwd_varlen with test and debug aids: a record
+ * of the mask the kernel actually applied, and stall injection for the
+ * bounded device-side waits.  Same arguments as attn_fwd_varlen plus `dbg`.
+ * It runs a separate instantiation of the attention kernel, compiled from the
+ * same source with these aids added; results in `o` are those of
+ * attn_fwd_varlen.  Adjacent RoPE pairs only (RKV_ERR_UNSUPPORTED otherwise).
+ *
+ * Mask record.  The frame-block-causal mask ("Amazon and Reactor tune
+ * Trainium for real-time video generation", section "Three problems for
+ * generic compilers": two passes per window with different attention
+ * lengths) is applied on the device by the choice of key tiles a work unit
+ * processes and by a per-element predicate on partial tiles.  With row_stats
+ * set, every softmax thread counts, after that masking, the scores of its
+ * query row that are not -inf (every other score of N(0,1)-sized inputs is
+ * finite), and writes for (sequence i in the order given, query row r, head h)
+ * at int32 index 4 * ((Lq_0 + ... + Lq_{i-1} + r) * H + h):
+ *   [0] keys that entered the softmax, [1] the sum of their key indices
+ *   (mod 2^32), [2] 1 + the largest such key index (0 if none),
+ *   [3] 128-key tiles the row's work unit processed
+ * (the two halves of a split tail unit add into one record).  For a row that
+ * sees exactly the keys [0, n): n, n(n-1)/2, n, ceil(n/128).
+ *
+ * Index checks.  The debug instantiation also checks, before each global
+ * store and TMA load it issues, the indices it computed against the launch's
+ * shapes (head < H, query row < Lq, key tile inside [0, Lk), split-unit slot
+ * inside the workspace); a failed check skips the store and records
+ * RKV_ERR_DEVICE_CHECK in the workspace (rkv_attn_status reports it).  Nothing
+ * traps.
+ *
+ * Stall injection (a test of the bounded waits that faults nothing): the
+ * second CTA of the first CTA pair withholds one handoff, so the pair's MMA
+ * issuer waits for it until the time limit, the kernel stops early and
+ * records RKV_ERR_TIMEOUT in the workspace (rkv_attn_status reports it).
+ * The outputs of that launch are then incomplete; the device stays usable.
+ *
+ *   dbg->row_stats   device int32 [(Lq_0 + ... + Lq_{n-1}) * H][4], 16-byte
+ *                    aligned, or NULL (no record); zeroed by the call
+ *   dbg->stall       RKV_DEBUG_STALL_NONE or one of the handoffs below
+ *   dbg->timeout_us  limit of every device-side wait of this launch in
+ *                    microseconds (0 = the default 2 s)
+ * Errors: those of attn_fwd_varlen, plus RKV_ERR_INVALID_ARG for a NULL dbg,
+ * an unknown stall or a misaligned row_stats.
+ */
+#define RKV_DEBUG_STALL_NONE 0u
+#define RKV_DEBUG_STALL_V_READY 1u /* its first "V tile landed" arrive          */
+#define RKV_DEBUG_STALL_K_READY 2u /* its first "K tile rotated" arrive         */
+#define RKV_DEBUG_STALL_P_FULL 3u  /* its first softmax warp's first "P ready"  */
+
+typedef struct {
+  int32_t* row_stats;
+  uint32_t stall;
+  uint32_t timeout_us;
+} rkv_attn_debug;
+
+rkv_status attn_fwd_varlen_debug(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                 float softmax_scale, const rkv_rope3d* rope, void* workspace,
+                                 size_t workspace_bytes, const rkv_attn_debug* dbg, void* stream);
 
 /*
  * attn_fwd_varlen_noalloc -- attn_fwd_varlen without a caller workspace.
@@ -244,12 +303,20 @@ rkv_status rkv_attn_status(void* workspace, void* stream);
  * and can be a few percent slower on full-size work; a launch whose minimum
  * scratch need exceeded the array would be rejected with
  * RKV_ERR_UNSUPPORTED.
- * A device-side timeout stops the kernel as in attn_fwd_varlen but is only
- * recorded in the internal array; callers that need it reported back use
- * attn_fwd_varlen with their own workspace and rkv_attn_status.
+ * A device-side timeout stops the kernel as in attn_fwd_varlen and is
+ * recorded in the internal array; rkv_attn_noalloc_status reads it back.
  */
 rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
                                    float softmax_scale, const rkv_rope3d* rope, void* stream);
+
+/*
+ * rkv_attn_noalloc_status -- rkv_attn_status for attn_fwd_varlen_noalloc:
+ * synchronise `stream`, return the status word the last no-alloc launch on
+ * the current device left in the library's internal array (RKV_OK or
+ * RKV_ERR_TIMEOUT) and clear it.  Allocates nothing; like the launch it reads,
+ * the first call on a device looks up the array's address.
+ */
+rkv_status rkv_attn_noalloc_status(void* stream);
 
 /*
  * Per-layer rolling KV cache.
@@ -309,7 +376,8 @@ typedef struct {
  * no bytes move for eviction.
  * The copy runs on the TMA bulk-copy engine; each of its waits on a bulk
  * load is bounded (1 s), after which the kernel stops, sets a per-GPU flag and
- * the insert is incomplete: rkv_ring_status reads that flag.
+ * the insert is incomplete (its destination slots may be partly written):
+ * rkv_ring_status reads that flag.
  * Errors: RKV_ERR_INVALID_ARG (n_frames above capacity or < 0, null
  * pointers, pinned/head/count out of range or inconsistent, D != 128,
  * misalignment, overlap).
@@ -345,6 +413,29 @@ rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_
 rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
                                     int64_t new_row_stride, int32_t n_frames, int32_t t0,
                                     const rkv_rope3d* rope, int32_t* n_evicted, void* stream);
+
+/*
+ * kvcache_ring_update_debug -- kvcache_ring_update with stall injection, a
+ * test of the copy's bounded waits that faults nothing.  Same arguments plus
+ * `dbg`; with dbg->stall = RKV_DEBUG_STALL_BULK_LOAD the first CTA declares
+ * 16 bytes more for its first piece than it loads, so that piece's wait runs
+ * out after dbg->timeout_us microseconds (0 = the default 1 s): the copy stops
+ * early, sets the flag rkv_ring_status reports, and the insert is incomplete
+ * (head and count still advance, as for a normal insert).  With
+ * RKV_DEBUG_STALL_NONE it is kvcache_ring_update with that wait limit.
+ * Errors: those of kvcache_ring_update, plus RKV_ERR_INVALID_ARG for a NULL
+ * dbg or an unknown stall.
+ */
+#define RKV_DEBUG_STALL_BULK_LOAD 1u
+
+typedef struct {
+  uint32_t stall;
+  uint32_t timeout_us;
+} rkv_ring_debug;
+
+rkv_status kvcache_ring_update_debug(rkv_ring* ring, const void* k_new, const void* v_new,
+                                     int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
+                                     const rkv_ring_debug* dbg, void* stream);
 
 /*
  * rkv_ring_status -- synchronise `stream` and report whether a ring insert on

@@ -58,7 +58,6 @@
 #include <utility>
 
 #include "common.cuh"
-#include "exp2_fma.cuh"
 #include "sm100_ptx.cuh"
 
 namespace rkv {
@@ -83,9 +82,6 @@ constexpr int kThreads = 16 * 32;
 constexpr int kTabEntryBytes = 32;   // cos and sin of 4 consecutive rotary pairs
 constexpr int kMaxTabEntries = 768;  // 24 KB of shared memory (cos array, then sin array)
 constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growth
-// Route one exponential pair in four to the FMA pipe.  Off: measured slower
-// on B200 at this kernel's operating point (the softmax is not MUFU-bound).
-constexpr bool kPolyExp = false;
 // register split (setmaxnreg): two softmax warpgroups, RoPE, producers; the
 // four shares add up to the 4 x 128 registers per thread the block launches with
 constexpr int kRegSoftmax = 176, kRegRope = 80, kRegProducer = 80;
@@ -113,6 +109,7 @@ struct SeqDev {
   uint32_t flags;
   int32_t n_qblocks;
   int32_t unit_begin;
+  int64_t stats_row0;   // debug launches: first row of this sequence in row_stats
 };
 
 struct Params {
@@ -137,12 +134,16 @@ struct Params {
   // axis of its first pair (lo) and of its last pair (hi); axes; and which
   // of the 4 pairs take the hi axis (0 when the chunk lies on one axis)
   int32_t ch_base_lo[16], ch_base_hi[16];
-  int8_t ch_ax_lo[16], ch_ax_hi[16], ch_sel[16];
+  int8_t ch_ax_lo[16], ch_ax_hi[16];
   uint32_t F;
   FastDiv div_F, div_W;
   double log2_theta[3];   // frequency base per axis (t, h, w)
   int32_t* status;
   uint64_t timeout_ns;
+  // debug launches only (attn_fwd_varlen_debug): per (row, head) mask record
+  // [4] int32 or null, and the handoff to skip (RKV_DEBUG_STALL_*)
+  int32_t* row_stats;
+  uint32_t stall;
 };
 
 // barrier indices.  The first group is used in every CTA; the second only in
@@ -196,6 +197,45 @@ __device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t b, uint32_t par
   return __all_sync(0xffffffffu, ok);
 }
 
+// After the CTA stopped: wait (bounded, without looking at the stop flag) for
+// a TMA load this thread issued to land, so no copy still writes this CTA's
+// shared memory when it exits.
+__device__ __forceinline__ void drain_phase(const Ctx& c, uint32_t b, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(b, parity))
+    if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) return;
+}
+
+// Debug launches: an index check; a failed one records RKV_ERR_DEVICE_CHECK
+// (and where) in the status word and returns false so the access is skipped.
+__device__ __forceinline__ bool dev_check(const Params& p, bool ok, int where) {
+  if (!ok) atomicCAS(p.status, 0, int(RKV_ERR_DEVICE_CHECK) | (where << 8));
+  return ok;
+}
+
+// Debug launches: one query row's record of the keys that entered its
+// softmax with a finite score (count, sum of key indices, 1 + largest index)
+// and of the key tiles it processed.
+struct RowStats {
+  uint32_t count, sum, top, tiles;
+};
+
+// Count the scores of one thread's row of a 128-key tile (first key kbase)
+// that are not -inf after masking: what the softmax actually sees.
+__device__ __forceinline__ void row_stats_tile(const uint32_t (&sr)[4][32], uint32_t kbase, RowStats& st) {
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const bool vis = sr[ch][i] != 0xFF800000u;
+      const uint32_t idx = kbase + uint32_t(ch * 32 + i);
+      st.count += vis ? 1u : 0u;
+      st.sum += vis ? idx : 0u;
+      st.top = vis ? idx + 1u : st.top;
+    }
+  st.tiles += 1u;
+}
+
 struct Unit {
   int si, head, qb, nkt;
   int kt0, kt1;   // key tiles [kt0, kt1) of this work item
@@ -245,10 +285,6 @@ __host__ __device__ __forceinline__ Unit decode_unit(const Params& p, int item) 
     else r.kt1 = r.nkt / 2;
   }
   return r;
-}
-
-__device__ __forceinline__ int axis_of(const Params& p, int pair) {
-  return pair < p.ax_first[1] ? 0 : (pair < p.ax_first[2] ? 1 : 2);
 }
 
 __device__ __forceinline__ int pick3(int a, int x, int y, int z) { return a == 0 ? x : (a == 1 ? y : z); }
@@ -422,9 +458,7 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 
 // P = exp2(S * scale_log2 - m_use) for one thread's row of S (in registers),
 // written as bf16 over the first 64 TMEM columns of the S region; returns the
-// row sum of the fp32 P.  kPoly: one pair in four takes the FMA-pipe exp2 (not
-// in masked tiles, whose hidden scores are -inf).
-template <bool kPoly>
+// row sum of the fp32 P.
 __device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uint32_t tS, float scale_log2,
                                                 float m_use) {
   const float2 sc2 = make_float2(scale_log2, scale_log2);
@@ -437,11 +471,7 @@ __device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uin
     for (int i = 0; i < 16; ++i) {
       const float2 x =
           __ffma2_rn(make_float2(__uint_as_float(sr[ch][2 * i]), __uint_as_float(sr[ch][2 * i + 1])), sc2, nm2);
-      float2 pp;
-      if (kPoly && (i & 3) == 3)
-        pp = rkv::exp2_fma2(x);
-      else
-        pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));  // exp2(-inf) = 0 for hidden keys
+      const float2 pp = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));  // exp2(-inf) = 0: hidden keys
       acc[i & 3] = __fadd2_rn(acc[i & 3], pp);
       pk[i] = pack_bf16x2(pp.x, pp.y);
     }
@@ -451,7 +481,7 @@ __device__ __forceinline__ float exp_store_tile(const uint32_t (&sr)[4][32], uin
   return (a01.x + a01.y) + (a23.x + a23.y);
 }
 
-// exp_store_tile<false> that also returns the row max of the raw scores in
+// exp_store_tile that also returns the row max of the raw scores in
 // mx: the exponentials use the running max m_use and are kept unless the
 // tile's own max exceeds it by more than the rescale threshold.
 __device__ __forceinline__ float exp_store_tile_max(const uint32_t (&sr)[4][32], uint32_t tS, float scale_log2,
@@ -500,8 +530,11 @@ __device__ __forceinline__ void setmaxnreg_dec_producer() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
 }
 
-// kPT/kPH: compile-time RoPE axis split (pairs on t and h), or 0/0 for any split
-template <int kPT, int kPH, bool kHalf>
+// kPT/kPH: compile-time RoPE axis split (pairs on t and h), or 0/0 for any split.
+// kDebug: the instantiation behind attn_fwd_varlen_debug, which also records
+// per-row mask statistics and can skip one handoff (stall injection); the
+// production instantiations compile neither.
+template <int kPT, int kPH, bool kHalf, bool kDebug>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -596,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int qrow = un.qb * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
       const int64_t my_limit = row_kv_limit(s, p, qrow < s.Lq ? qrow : s.Lq - 1);
       float m = -INFINITY, l = 0.f;
+      RowStats rs = {0u, 0u, 0u, 0u};
       for (int j = un.kt0; j < un.kt1; ++j, ++g) {
         if (!wait_warp(c, bar(c, B_SFULL + wg), g & 1u, 1)) goto done;
         ptx::tc_fence_after();
@@ -605,7 +639,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ptx::tmem_wait_ld();
         const int64_t kbase = int64_t(j) * kBN;
         const int lim = kbase + kBN > my_limit ? int(my_limit - kbase) : kBN;
+        // partial tile for some row of the warp: hide keys at or past each
+        // row's limit (the keys of a row's mask are a prefix)
         const bool masked = __any_sync(0xffffffffu, lim < kBN);
+        if (masked) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
+        }
+        if constexpr (kDebug) row_stats_tile(sr, uint32_t(kbase), rs);
         const float m_old = m;
         float m_new, tile_sum;
         bool need;
@@ -618,16 +662,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           need = m_new > m + kRescaleLog2;
           if (__any_sync(0xffffffffu, need)) {
             if (need) m = m_new;
-            tile_sum = exp_store_tile<false>(sr, tS, scale_log2, m);
+            tile_sum = exp_store_tile(sr, tS, scale_log2, m);
           }
         } else {
-          if (masked) {
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
-          }
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
@@ -639,8 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           need = m_new > m + kRescaleLog2;
           if (need) m = m_new;
           const float m_use = (m == -INFINITY) ? 0.f : m;
-          tile_sum = masked ? exp_store_tile<false>(sr, tS, scale_log2, m_use)
-                            : exp_store_tile<kPolyExp>(sr, tS, scale_log2, m_use);
+          tile_sum = exp_store_tile(sr, tS, scale_log2, m_use);
         }
         if (j > un.kt0 && __any_sync(0xffffffffu, need)) {
           // O holds tiles 0..j-1 scaled to the old max: wait for the last PV,
@@ -663,7 +699,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(pfull);
+        bool skip = false;
+        if constexpr (kDebug)   // stall injection: the peer CTA's first softmax warp withholds its first P
+          skip = p.stall == RKV_DEBUG_STALL_P_FULL && cluster == 0 && rank == 1 && warp == 0 && g == 0;
+        if (lane == 0 && !skip) ptx::mbar_arrive_cluster(pfull);
       }
       // epilogue: O / l -> bf16 -> global (row-major [Lq][H][128])
       if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 3)) goto done;
@@ -678,7 +717,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(ofree);   // O may now be overwritten
-        if (un.part >= 0) {
+        bool store_ok = true;
+        if constexpr (kDebug) {
+          store_ok = dev_check(p, un.head >= 0 && un.head < p.H, 40);
+          if (un.part >= 0)
+            store_ok &= dev_check(p, un.part < 2 * p.n_split, 41);
+          else if (qrow < s.Lq)
+            store_ok &= dev_check(p, qrow >= 0 && int64_t(qrow) * s.o_stride_bytes + int64_t(un.head + 1) * (kHD * 2) <=
+                                             int64_t(s.Lq - 1) * s.o_stride_bytes + int64_t(p.H) * (kHD * 2), 42);
+          if (p.row_stats && qrow < s.Lq) {
+            // the two halves of a split unit add up into the same record
+            int32_t* rec = p.row_stats + ((s.stats_row0 + qrow) * p.H + un.head) * 4;
+            atomicAdd(reinterpret_cast<unsigned*>(rec + 0), rs.count);
+            atomicAdd(reinterpret_cast<unsigned*>(rec + 1), rs.sum);
+            atomicMax(reinterpret_cast<unsigned*>(rec + 2), rs.top);
+            atomicAdd(reinterpret_cast<unsigned*>(rec + 3), rs.tiles);
+          }
+        }
+        if (!store_ok) {
+        } else if (un.part >= 0) {
           // half of a split unit: unnormalised O, running max and row sum
           // for the combine pass
           const int64_t prow = int64_t(un.part) * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
@@ -714,8 +771,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
       const Unit un = decode_unit(p, u);
       const SeqDev& s = p.seq[un.si];
-      if (!wait_warp(c, bar(c, B_QFULL), ul & 1u, 4)) goto done;
-      if (s.flags & RKV_ROPE_Q) {
+      // Every RoPE warp reaches the named barrier below, whether its own wait
+      // succeeded or not, and the barrier's AND takes the stop decision for
+      // all four: a warp that left alone would hold the others at it.
+      const bool okq = wait_warp(c, bar(c, B_QFULL), ul & 1u, 4);
+      if (okq && (s.flags & RKV_ROPE_Q)) {
         // thread rt rotates row rt of both Q sub-tiles (all 16 chunks)
         for (int b = 0; b < kSub; ++b) {
           const int row = un.qb * kUnitRows + int(rank) * kCtaRows + b * kBM + rt;
@@ -732,12 +792,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
       }
       ptx::fence_proxy_async_smem();
-      ptx::named_sync(1, 128);
+      if (!ptx::named_sync_and(1, 128, okq)) goto done;
       if (rt == 0) ptx::mbar_arrive_cluster(qready);
       for (int j = un.kt0; j < un.kt1; ++j, ++it) {
         const uint32_t st = it % kStages, n = it / kStages;
-        if (!wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5)) goto done;
-        if (s.flags & RKV_ROPE_K) {
+        const bool okk = wait_warp(c, bar(c, B_KFULL + st), n & 1u, 5);
+        if (okk && (s.flags & RKV_ROPE_K)) {
           // this CTA's 64 keys of the tile: two threads per key row, warps
           // 8-9 take chunks 0-7 (first 64 columns), warps 10-11 chunks 8-15
           const int r = rt & 63;
@@ -760,8 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           }
         }
         ptx::fence_proxy_async_smem();
-        ptx::named_sync(1, 128);
-        if (rt == 0) ptx::mbar_arrive_cluster(lbar(B_KREADY + st));
+        if (!ptx::named_sync_and(1, 128, okk)) goto done;
+        bool skip = false;
+        if constexpr (kDebug)   // stall injection: the peer CTA withholds its first rotated K tile
+          skip = p.stall == RKV_DEBUG_STALL_K_READY && cluster == 0 && rank == 1 && it == 0;
+        if (rt == 0 && !skip) ptx::mbar_arrive_cluster(lbar(B_KREADY + st));
       }
     }
   } else {
@@ -773,16 +836,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ptx::tma_prefetch_desc(&p.seq[i].tk);
       }
       uint32_t it = 0, ul = 0;
+      bool ok = true;
       for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
         const Unit un = decode_unit(p, u);
         const SeqDev& s = p.seq[un.si];
-        if (!wait_phase(c, bar(c, B_QFREE), (ul & 1u) ^ 1u, 6)) break;
+        if (!wait_phase(c, bar(c, B_QFREE), (ul & 1u) ^ 1u, 6)) { ok = false; break; }
+        if constexpr (kDebug) {
+          dev_check(p, un.head >= 0 && un.head < p.H && un.qb >= 0 && int64_t(un.qb) * kUnitRows < s.Lq, 43);
+          dev_check(p, un.kt0 >= 0 && un.kt0 < un.kt1 && int64_t(un.kt1 - 1) * kBN < s.Lk, 44);
+        }
         ptx::mbar_expect_tx(bar(c, B_QFULL), kSub * kQTileBytes);
         for (int b = 0; b < kSub; ++b)
           for (int h2 = 0; h2 < 2; ++h2)
             ptx::tma_load_3d(sQ + b * kQTileBytes + h2 * kQHalfBytes, &s.tq, bar(c, B_QFULL), h2 * 64, un.head,
                              un.qb * kUnitRows + int(rank) * kCtaRows + b * kBM);
-        bool ok = true;
         for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_KFREE + st), (n & 1u) ^ 1u, 7)) { ok = false; break; }
@@ -791,7 +858,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             ptx::tma_load_3d(sK + st * kKStageBytes + h2 * kKHalfBytes, &s.tk, bar(c, B_KFULL + st), h2 * 64,
                              un.head, j * kBN + int(rank) * kKRows);
         }
-        if (!ok) break;
+        if (!ok) { ++ul; break; }
+      }
+      if (!ok) {
+        // stopped early: let this thread's last Q load and K loads land
+        if (ul > 0) drain_phase(c, bar(c, B_QFULL), (ul - 1) & 1u);
+        for (uint32_t i = it > uint32_t(kStages) ? it - kStages : 0u; i < it; ++i)
+          drain_phase(c, bar(c, B_KFULL + i % kStages), (i / kStages) & 1u);
       }
     } else if (warp == 14 && lane == 0) {
       // ===================== TMA producer: this CTA's V column half =====================
@@ -808,6 +881,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::tma_load_3d(sV + st * kVStageBytes, &s.tv, bar(c, B_VFULL + st), int(rank) * 64, un.head, j * kBN);
         }
       }
+      if (!ok) {
+        // stopped early: let this thread's last V loads land
+        for (uint32_t i = it > uint32_t(kStages) ? it - kStages : 0u; i < it; ++i)
+          drain_phase(c, bar(c, B_VFULL + i % kStages), (i / kStages) & 1u);
+      }
     } else if (warp == 15 && lane == 0) {
       // ===================== V landed -> tell the leader =====================
       uint32_t it = 0;
@@ -817,7 +895,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_VFULL + st), n & 1u, 17)) { ok = false; break; }
-          ptx::mbar_arrive_cluster(lbar(B_VREADY + st));
+          bool skip = false;
+          if constexpr (kDebug)   // stall injection: the peer CTA withholds its first V tile
+            skip = p.stall == RKV_DEBUG_STALL_V_READY && cluster == 0 && rank == 1 && it == 0;
+          if (!skip) ptx::mbar_arrive_cluster(lbar(B_VREADY + st));
         }
       }
     } else if (warp == 13 && lane == 0 && rank == 0) {
@@ -1014,15 +1095,17 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __g
 // Launch shape of the attention kernel (attributes set, cluster of 2) and the
 // number of clusters that fit on the current device at once.
 // Kernel instantiation: the pages' 22/21/21 split gets a compile-time axis
-// map (either pair layout); other splits read it from the parameters.
-static void (*attn_kernel_for(bool default_split, bool half))(Params) {
-  if (half) return default_split ? attn_fwd_kernel<22, 21, true> : attn_fwd_kernel<0, 0, true>;
-  return default_split ? attn_fwd_kernel<22, 21, false> : attn_fwd_kernel<0, 0, false>;
+// map (either pair layout); other splits read it from the parameters.  Debug
+// launches (adjacent pairs only) use the kDebug instantiations.
+static void (*attn_kernel_for(bool default_split, bool half, bool debug))(Params) {
+  if (debug) return default_split ? attn_fwd_kernel<22, 21, false, true> : attn_fwd_kernel<0, 0, false, true>;
+  if (half) return default_split ? attn_fwd_kernel<22, 21, true, false> : attn_fwd_kernel<0, 0, true, false>;
+  return default_split ? attn_fwd_kernel<22, 21, false, false> : attn_fwd_kernel<0, 0, false, false>;
 }
 
-static rkv_status attn_launch_shape(bool default_split, bool half, cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr,
-                                    const void*& kern_ptr, int& max_clusters) {
-  auto kern = attn_kernel_for(default_split, half);
+static rkv_status attn_launch_shape(bool default_split, bool half, bool debug, cudaLaunchConfig_t& cfg,
+                                    cudaLaunchAttribute* attr, const void*& kern_ptr, int& max_clusters) {
+  auto kern = attn_kernel_for(default_split, half, debug);
   kern_ptr = reinterpret_cast<const void*>(kern);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
@@ -1067,7 +1150,7 @@ extern "C" size_t attn_fwd_varlen_workspace_size(const rkv_attn_seq*, int32_t, i
   cudaLaunchAttribute attr[1];
   const void* kern = nullptr;
   int clusters = 0;
-  if (attn_launch_shape(true, false, cfg, attr, kern, clusters) != RKV_OK) {
+  if (attn_launch_shape(true, false, false, cfg, attr, kern, clusters) != RKV_OK) {
     clear_error();
     return kWorkspaceBytes;
   }
@@ -1105,9 +1188,12 @@ static int64_t plan_units(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, i
   for (int i = 1; i < n_seqs; ++i)
     for (int j = i; j > 0 && seqs[order[j]].Lk > seqs[order[j - 1]].Lk; --j) std::swap(order[j], order[j - 1]);
   int64_t units = 0;
+  int64_t row0[RKV_MAX_SEQS];
+  for (int i = 0, r = 0; i < n_seqs; r += seqs[i].Lq, ++i) row0[i] = r;
   for (int oi = 0; oi < n_seqs; ++oi) {
     const rkv_attn_seq& s = seqs[order[oi]];
     SeqDev& d = p.seq[oi];
+    d.stats_row0 = row0[order[oi]];
     d.Lq = s.Lq; d.Lk = s.Lk; d.q_t0 = s.q_t0; d.k_t0 = s.k_t0;
     d.q_frame_offset = s.q_frame_offset; d.block_frames = s.block_frames; d.flags = s.flags;
     d.n_qblocks = (s.Lq + kUnitRows - 1) / kUnitRows;   // 512-row blocks, one per CTA pair
@@ -1121,10 +1207,11 @@ static int64_t plan_units(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, i
   return units;
 }
 
-extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
-                                      float softmax_scale, const rkv_rope3d* rope, void* workspace,
-                                      size_t workspace_bytes, void* stream) {
-  clear_error();
+// Checks, plans and launches one attention call (dbg = null for the
+// production entry points).
+static rkv_status attn_launch(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D, float softmax_scale,
+                              const rkv_rope3d* rope, void* workspace, size_t workspace_bytes,
+                              const rkv_attn_debug* dbg, void* stream) {
   if (!seqs || n_seqs < 1) return fail(RKV_ERR_INVALID_ARG, "need at least one sequence");
   if (n_seqs > RKV_MAX_SEQS) return fail(RKV_ERR_UNSUPPORTED, "at most %d sequences per launch", RKV_MAX_SEQS);
   if (H < 1) return fail(RKV_ERR_INVALID_ARG, "H must be >= 1");
@@ -1206,10 +1293,6 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
     p.ch_ax_hi[g] = int8_t(ahi);
     p.ch_base_lo[g] = p.ax_tab[alo] + (g - p.ax_chunk0[alo]) * p.ax_npos[alo];
     p.ch_base_hi[g] = p.ax_tab[ahi] + (g - p.ax_chunk0[ahi]) * p.ax_npos[ahi];
-    int sel = 0;
-    if (ahi != alo)
-      for (int j = 0; j < 4; ++j) sel |= (axis_of_pair(4 * g + j) == ahi) << j;
-    p.ch_sel[g] = int8_t(sel);
   }
   p.n_seqs = n_seqs;
   p.H = H;
@@ -1225,6 +1308,11 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   p.log2_theta[2] = log2(double(rope->theta_w != 0.0f ? rope->theta_w : rope->theta));
   p.status = static_cast<int32_t*>(workspace);
   p.timeout_ns = 2000000000ull;
+  if (dbg) {   // checked by attn_fwd_varlen_debug
+    if (dbg->timeout_us > 0) p.timeout_ns = uint64_t(dbg->timeout_us) * 1000ull;
+    p.row_stats = dbg->row_stats;
+    p.stall = dbg->stall;
+  }
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // the 22/21/21 split of the pages' 128-dim heads gets its own instantiation
@@ -1234,7 +1322,8 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   const void* kern = nullptr;
   int max_clusters = 0;
   const bool half = rope->layout == RKV_ROPE_HALF;
-  if ((st = attn_launch_shape(default_split, half, cfg, attr, kern, max_clusters)) != RKV_OK) return st;
+  if ((st = attn_launch_shape(default_split, half, dbg != nullptr, cfg, attr, kern, max_clusters)) != RKV_OK)
+    return st;
   cfg.stream = cs;
 
   // tail split: the last n_split units run as two half-units each when the
@@ -1274,9 +1363,15 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
 
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWorkspaceBytes, cs);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  if (p.row_stats) {
+    int64_t rows = 0;
+    for (int i = 0; i < n_seqs; ++i) rows += seqs[i].Lq;
+    e = cudaMemsetAsync(p.row_stats, 0, size_t(rows) * H * 4 * sizeof(int32_t), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(row_stats)");
+  }
   // one CTA pair per pair of SMs that can hold it (persistent)
   cfg.gridDim = dim3(uint32_t(2 * std::min<int64_t>(p.total_units, max_clusters)));
-  e = cudaLaunchKernelEx(&cfg, attn_kernel_for(default_split, half), p);
+  e = cudaLaunchKernelEx(&cfg, attn_kernel_for(default_split, half, dbg != nullptr), p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   if (n_split > 0) {
@@ -1288,9 +1383,31 @@ extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, 
   return RKV_OK;
 }
 
+extern "C" rkv_status attn_fwd_varlen(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                      float softmax_scale, const rkv_rope3d* rope, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("attn_fwd_varlen");
+  clear_error();
+  return attn_launch(seqs, n_seqs, H, D, softmax_scale, rope, workspace, workspace_bytes, nullptr, stream);
+}
+
+extern "C" rkv_status attn_fwd_varlen_debug(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
+                                            float softmax_scale, const rkv_rope3d* rope, void* workspace,
+                                            size_t workspace_bytes, const rkv_attn_debug* dbg, void* stream) {
+  NvtxRange nvtx_range("attn_fwd_varlen_debug");
+  clear_error();
+  if (!dbg) return fail(RKV_ERR_INVALID_ARG, "debug settings are NULL");
+  if (dbg->stall > RKV_DEBUG_STALL_P_FULL) return fail(RKV_ERR_INVALID_ARG, "unknown debug stall %u", dbg->stall);
+  if (dbg->row_stats && !aligned16(dbg->row_stats)) return fail(RKV_ERR_INVALID_ARG, "row_stats must be 16-byte aligned");
+  if (rope && rope->layout != RKV_ROPE_ADJACENT)
+    return fail(RKV_ERR_UNSUPPORTED, "debug launches support the adjacent RoPE pair layout only");
+  return attn_launch(seqs, n_seqs, H, D, softmax_scale, rope, workspace, workspace_bytes, dbg, stream);
+}
+
 extern "C" rkv_status rkv_attn_mask_rows(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H,
                                          const rkv_rope3d* rope, int64_t* row_limit, int32_t* unit_tiles,
                                          int64_t* n_units) {
+  NvtxRange nvtx_range("rkv_attn_mask_rows");
   clear_error();
   if (!seqs || n_seqs < 1) return fail(RKV_ERR_INVALID_ARG, "need at least one sequence");
   if (n_seqs > RKV_MAX_SEQS) return fail(RKV_ERR_UNSUPPORTED, "at most %d sequences per launch", RKV_MAX_SEQS);
@@ -1331,6 +1448,7 @@ extern "C" rkv_status rkv_attn_mask_rows(const rkv_attn_seq* seqs, int32_t n_seq
 }
 
 extern "C" rkv_status rkv_attn_status(void* workspace, void* stream) {
+  NvtxRange nvtx_range("rkv_attn_status");
   clear_error();
   if (!workspace) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -1342,6 +1460,8 @@ extern "C" rkv_status rkv_attn_status(void* workspace, void* stream) {
   e = cudaMemsetAsync(workspace, 0, sizeof(word), cs);
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the attention status word");
+  if ((word & 0xff) == RKV_ERR_DEVICE_CHECK)
+    return fail(RKV_ERR_DEVICE_CHECK, "attention debug launch: device-side index check %d failed", word >> 8);
   return fail(rkv_status(word & 0xff), "attention kernel stopped: bounded wait %d timed out", word >> 8);
 }
 
@@ -1388,6 +1508,7 @@ static rkv_status noalloc_scratch(void** out) {
 
 extern "C" rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t H, int32_t D,
                                               float softmax_scale, const rkv_rope3d* rope, void* stream) {
+  NvtxRange nvtx_range("attn_fwd_varlen_noalloc");
   clear_error();
   // the launch needs kWorkspaceBytes at least; with no room for partial
   // results it runs without the tail split
@@ -1398,5 +1519,14 @@ extern "C" rkv_status attn_fwd_varlen_noalloc(const rkv_attn_seq* seqs, int32_t 
   void* ws = nullptr;
   rkv_status st = noalloc_scratch(&ws);
   if (st != RKV_OK) return st;
-  return attn_fwd_varlen(seqs, n_seqs, H, D, softmax_scale, rope, ws, kNoAllocScratchBytes, stream);
+  return attn_launch(seqs, n_seqs, H, D, softmax_scale, rope, ws, kNoAllocScratchBytes, nullptr, stream);
+}
+
+extern "C" rkv_status rkv_attn_noalloc_status(void* stream) {
+  NvtxRange nvtx_range("rkv_attn_noalloc_status");
+  clear_error();
+  void* ws = nullptr;
+  rkv_status st = noalloc_scratch(&ws);
+  if (st != RKV_OK) return st;
+  return rkv_attn_status(ws, stream);
 }

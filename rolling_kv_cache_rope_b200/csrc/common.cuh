@@ -3,11 +3,22 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "rkv.h"
 
 namespace rkv {
+
+// ---- host: an NVTX range around each entry point, so a profiler's timeline
+// shows which library call enqueued which kernels (a no-op when no tool is
+// attached) ----
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ---- host: per-thread last-error text ------------------------------------
 void set_error(const char* fmt, ...);
@@ -90,7 +101,6 @@ inline FastDiv make_fastdiv(uint32_t d) {
 __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
   return (__umulhi(n, f.m) + n) >> f.s;
 }
-__device__ __forceinline__ uint32_t fmod_(uint32_t n, uint32_t q, const FastDiv& f) { return n - q * f.d; }
 
 // ---- bf16 packing -----------------------------------------------------------
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t u) { return __uint_as_float(u << 16); }

@@ -10,7 +10,7 @@ namespace rkv {
 
 constexpr int kBulkStages = 6;                      // most pieces in flight per CTA
 constexpr uint32_t kBulkStageBytes = 32768;         // largest piece
-constexpr uint64_t kBulkWaitNs = 1000000000ull;     // 1 s per wait, then give up
+constexpr uint64_t kBulkWaitNs = 1000000000ull;     // default limit of one wait (1 s), then give up
 
 // Pieces of an insert: the K pieces first, then the V pieces; within a
 // tensor, frame by frame, each frame as groups of rpp whole rows (or, when one
@@ -33,6 +33,8 @@ struct RingBulkArgs {
   uint32_t contiguous;      // source rows are back to back (one load per piece)
   RingPlan plan;            // destination slot of each frame
   int32_t* timeout_flag;    // set to 1 when a wait gives up
+  uint64_t wait_ns;         // limit of one wait
+  uint32_t stall;           // debug: CTA 0 declares 16 bytes more for its first piece than it loads
 };
 
 struct RingPiece {
@@ -61,21 +63,22 @@ __device__ __forceinline__ RingPiece ring_piece(const RingBulkArgs& a, uint32_t 
   return pc;
 }
 
-// Bounded wait (at most kBulkWaitNs) for the phase of `bar` with parity
+// Bounded wait (at most limit_ns) for the phase of `bar` with parity
 // `parity` to complete.
-__device__ __forceinline__ bool bulk_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool bulk_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (!ptx::mbar_try_wait(bar, parity))
-    if (ptx::globaltimer_ns() - t0 > kBulkWaitNs) return false;
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
   return true;
 }
 
 // Issue the bulk load(s) of piece pc into shared memory at dst, completing on
-// the mbarrier at bar.
+// the mbarrier at bar.  `extra` bytes are declared on top of what is loaded
+// (0 except for stall injection, which makes the barrier never complete).
 __device__ __forceinline__ void bulk_load_piece(const RingBulkArgs& a, const RingPiece& pc, uint32_t dst,
-                                                uint32_t bar) {
-  ptx::mbar_expect_tx(bar, pc.rows * pc.cols);
+                                                uint32_t bar, uint32_t extra = 0) {
+  ptx::mbar_expect_tx(bar, pc.rows * pc.cols + extra);
   if (a.contiguous) {
     ptx::bulk_load(dst, pc.src, pc.rows * pc.cols, bar);
   } else {
@@ -97,7 +100,8 @@ __device__ __forceinline__ RingPiece cta_piece(const RingBulkArgs& a, uint32_t i
   return ring_piece(a, blockIdx.x + i * gridDim.x);
 }
 
-// Piece geometry of an insert into a checked ring (all but timeout_flag).
+// Piece geometry of an insert into a checked ring (timeout_flag left null,
+// default wait limit, no stall).
 inline rkv_status ring_bulk_geometry(const rkv_ring* ring, const void* k_new, const void* v_new,
                                      int64_t new_row_stride, int32_t n_frames, RingBulkArgs& a) {
   a.src[0] = static_cast<const uint8_t*>(k_new);
@@ -129,6 +133,8 @@ inline rkv_status ring_bulk_geometry(const rkv_ring* ring, const void* k_new, co
   a.contiguous = a.src_row_stride == a.row_bytes ? 1u : 0u;
   a.plan = ring_plan(ring);
   a.timeout_flag = nullptr;
+  a.wait_ns = kBulkWaitNs;
+  a.stall = 0;
   return RKV_OK;
 }
 

@@ -39,10 +39,12 @@ __global__ void __launch_bounds__(kBulkThreads, 1) ring_bulk_kernel(const RingBu
   auto stage = [&](uint32_t i) { return smem0 + (i % a.stages) * a.stage_bytes; };
   auto bar = [&](uint32_t i) { return ptx::smem_u32(&full[i % a.stages]); };
   uint32_t issued = 0;
-  for (; issued < n && issued < a.stages; ++issued) bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued));
+  for (; issued < n && issued < a.stages; ++issued)
+    bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued),
+                    (a.stall && blockIdx.x == 0 && issued == 0) ? 16u : 0u);
   uint32_t i = 0;
   for (; i < n; ++i) {
-    if (!bulk_wait(bar(i), (i / a.stages) & 1u)) {
+    if (!bulk_wait(bar(i), (i / a.stages) & 1u, a.wait_ns)) {
       atomicExch(a.timeout_flag, 1);
       break;
     }
@@ -55,9 +57,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) ring_bulk_kernel(const RingBu
       ++issued;
     }
   }
-  // after a wait gave up: let the loads still in flight land (bounded) before
-  // the CTA's shared memory is released
-  for (uint32_t j = i + 1; j < issued; ++j) bulk_wait(bar(j), (j / a.stages) & 1u);
+  // after a wait gave up on piece i: let the loads still in flight, piece i's
+  // included, land (bounded) before the CTA's shared memory is released
+  // (issued <= i + stages, so these pieces use distinct stages)
+  for (uint32_t j = i; j < issued; ++j) bulk_wait(bar(j), (j / a.stages) & 1u, a.wait_ns);
   ptx::bulk_wait_all();
 }
 
@@ -160,10 +163,14 @@ static rkv_status ring_timeout_flag(int32_t** out) {
 // Host side of one insert: piece geometry, grid of one CTA per SM (or fewer
 // when the insert has fewer pieces), shared memory for the stages.
 static rkv_status launch_ring_bulk(const rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
-                                   int32_t n_frames, cudaStream_t stream) {
+                                   int32_t n_frames, const rkv_ring_debug* dbg, cudaStream_t stream) {
   RingBulkArgs a;
   rkv_status st = ring_bulk_geometry(ring, k_new, v_new, new_row_stride, n_frames, a);
   if (st != RKV_OK) return st;
+  if (dbg) {
+    if (dbg->timeout_us > 0) a.wait_ns = uint64_t(dbg->timeout_us) * 1000ull;
+    a.stall = dbg->stall;
+  }
   st = ring_timeout_flag(&a.timeout_flag);
   if (st != RKV_OK) return st;
   const int smem = int(a.stages * a.stage_bytes);
@@ -194,23 +201,40 @@ extern "C" int32_t rkv_ring_slot(const rkv_ring* ring, int32_t j) {
   return int32_t(P + s);
 }
 
-extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_new,
-                                          int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
-                                          void* stream) {
-  clear_error();
+static rkv_status ring_update(rkv_ring* ring, const void* k_new, const void* v_new, int64_t new_row_stride,
+                              int32_t n_frames, int32_t* n_evicted, const rkv_ring_debug* dbg, void* stream) {
   rkv_status st = check_ring(ring);
   if (st != RKV_OK) return st;
   st = check_ring_insert(ring, k_new, v_new, new_row_stride, n_frames);
   if (st != RKV_OK) return st;
   if (n_frames > 0) {
-    st = launch_ring_bulk(ring, k_new, v_new, new_row_stride, n_frames, static_cast<cudaStream_t>(stream));
+    st = launch_ring_bulk(ring, k_new, v_new, new_row_stride, n_frames, dbg, static_cast<cudaStream_t>(stream));
     if (st != RKV_OK) return st;
   }
   ring_advance(ring, n_frames, n_evicted);
   return RKV_OK;
 }
 
+extern "C" rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_new,
+                                          int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
+                                          void* stream) {
+  NvtxRange nvtx_range("kvcache_ring_update");
+  clear_error();
+  return ring_update(ring, k_new, v_new, new_row_stride, n_frames, n_evicted, nullptr, stream);
+}
+
+extern "C" rkv_status kvcache_ring_update_debug(rkv_ring* ring, const void* k_new, const void* v_new,
+                                                int64_t new_row_stride, int32_t n_frames, int32_t* n_evicted,
+                                                const rkv_ring_debug* dbg, void* stream) {
+  NvtxRange nvtx_range("kvcache_ring_update_debug");
+  clear_error();
+  if (!dbg) return fail(RKV_ERR_INVALID_ARG, "debug settings are NULL");
+  if (dbg->stall > RKV_DEBUG_STALL_BULK_LOAD) return fail(RKV_ERR_INVALID_ARG, "unknown debug stall %u", dbg->stall);
+  return ring_update(ring, k_new, v_new, new_row_stride, n_frames, n_evicted, dbg, stream);
+}
+
 extern "C" rkv_status rkv_ring_status(void* stream) {
+  NvtxRange nvtx_range("rkv_ring_status");
   clear_error();
   int32_t* flag = nullptr;
   rkv_status st = ring_timeout_flag(&flag);
@@ -224,5 +248,5 @@ extern "C" rkv_status rkv_ring_status(void* stream) {
   e = cudaMemsetAsync(flag, 0, sizeof(int32_t), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the ring timeout flag");
-  return fail(RKV_ERR_TIMEOUT, "a ring insert's bulk-copy wait gave up after 1 s; the insert is incomplete");
+  return fail(RKV_ERR_TIMEOUT, "a ring insert's bulk-copy wait gave up; the insert is incomplete");
 }

@@ -370,6 +370,7 @@ using namespace rkv;
 
 extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H, int32_t D, int64_t x_row_stride,
                                    int64_t y_row_stride, int32_t t0, const rkv_rope3d* rope, void* stream) {
+  NvtxRange nvtx_range("rope3d_apply");
   clear_error();
   if (D != 128) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", D);
   rkv_status st = check_rope(rope, D);
@@ -401,6 +402,7 @@ extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H,
 extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
                                                int64_t new_row_stride, int32_t n_frames, int32_t t0,
                                                const rkv_rope3d* rope, int32_t* n_evicted, void* stream) {
+  NvtxRange nvtx_range("kvcache_ring_update_rope");
   clear_error();
   rkv_status st = check_ring(ring);
   if (st != RKV_OK) return st;

@@ -21,11 +21,11 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-RKV_OK, RKV_ERR_INVALID_ARG, RKV_ERR_UNSUPPORTED, RKV_ERR_CUDA, RKV_ERR_TIMEOUT = 0, 1, 2, 3, 4
+RKV_OK, RKV_ERR_INVALID_ARG, RKV_ERR_UNSUPPORTED, RKV_ERR_CUDA, RKV_ERR_TIMEOUT, RKV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4, 5
 RKV_ROPE_Q, RKV_ROPE_K = 1, 2
 RKV_MAX_SEQS = 16
 STATUS_NAMES = {0: "RKV_OK", 1: "RKV_ERR_INVALID_ARG", 2: "RKV_ERR_UNSUPPORTED", 3: "RKV_ERR_CUDA",
-                4: "RKV_ERR_TIMEOUT"}
+                4: "RKV_ERR_TIMEOUT", 5: "RKV_ERR_DEVICE_CHECK"}
 
 
 class rkv_rope3d(ctypes.Structure):
@@ -45,6 +45,18 @@ class rkv_attn_seq(ctypes.Structure):
                 ("block_frames", ctypes.c_int32), ("flags", ctypes.c_uint32), ("reserved", ctypes.c_int32)]
 
 
+class rkv_attn_debug(ctypes.Structure):
+    _fields_ = [("row_stats", ctypes.c_void_p), ("stall", ctypes.c_uint32), ("timeout_us", ctypes.c_uint32)]
+
+
+class rkv_ring_debug(ctypes.Structure):
+    _fields_ = [("stall", ctypes.c_uint32), ("timeout_us", ctypes.c_uint32)]
+
+
+RKV_DEBUG_STALL_NONE, RKV_DEBUG_STALL_V_READY, RKV_DEBUG_STALL_K_READY, RKV_DEBUG_STALL_P_FULL = 0, 1, 2, 3
+RKV_DEBUG_STALL_BULK_LOAD = 1
+
+
 class rkv_ring(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("slots", ctypes.c_int32),
                 ("tokens_per_frame", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
@@ -62,6 +74,15 @@ _lib.attn_fwd_varlen.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int3
                                  _c.POINTER(rkv_rope3d), _c.c_void_p, _c.c_size_t, _c.c_void_p]
 _lib.rkv_attn_status.restype = _c.c_int
 _lib.rkv_attn_status.argtypes = [_c.c_void_p, _c.c_void_p]
+_lib.attn_fwd_varlen_debug.restype = _c.c_int
+_lib.attn_fwd_varlen_debug.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int32, _c.c_int32, _c.c_float,
+                                       _c.POINTER(rkv_rope3d), _c.c_void_p, _c.c_size_t, _c.POINTER(rkv_attn_debug),
+                                       _c.c_void_p]
+_lib.attn_fwd_varlen_noalloc.restype = _c.c_int
+_lib.attn_fwd_varlen_noalloc.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int32, _c.c_int32, _c.c_float,
+                                         _c.POINTER(rkv_rope3d), _c.c_void_p]
+_lib.rkv_attn_noalloc_status.restype = _c.c_int
+_lib.rkv_attn_noalloc_status.argtypes = [_c.c_void_p]
 _lib.rkv_attn_mask_rows.restype = _c.c_int
 _lib.rkv_attn_mask_rows.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int32, _c.POINTER(rkv_rope3d),
                                     _c.POINTER(_c.c_int64), _c.POINTER(_c.c_int32), _c.POINTER(_c.c_int64)]
@@ -71,6 +92,9 @@ _lib.kvcache_ring_update.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_voi
 _lib.kvcache_ring_update_rope.restype = _c.c_int
 _lib.kvcache_ring_update_rope.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
                                           _c.c_int32, _c.POINTER(rkv_rope3d), _c.POINTER(_c.c_int32), _c.c_void_p]
+_lib.kvcache_ring_update_debug.restype = _c.c_int
+_lib.kvcache_ring_update_debug.argtypes = [_c.POINTER(rkv_ring), _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32,
+                                           _c.POINTER(_c.c_int32), _c.POINTER(rkv_ring_debug), _c.c_void_p]
 _lib.rkv_ring_status.restype = _c.c_int
 _lib.rkv_ring_status.argtypes = [_c.c_void_p]
 _lib.rkv_ring_slot.restype = _c.c_int32
@@ -193,6 +217,52 @@ def rkv_attn_status(workspace, stream=None):
     _check(_lib.rkv_attn_status(workspace.data_ptr(), _stream(stream)))
 
 
+def attn_fwd_varlen_debug(seqs, rope, row_stats=None, stall=RKV_DEBUG_STALL_NONE, timeout_us=0, softmax_scale=None,
+                          workspace=None, stream=None):
+    """attn_fwd_varlen with test and debug aids (see rkv.h): ``row_stats`` an
+    int32 CUDA tensor of sum(Lq) * H * 4 elements that receives the per-row
+    mask record; ``stall`` one of RKV_DEBUG_STALL_*; ``timeout_us`` the limit
+    of every device-side wait (0 = default).  Returns the workspace."""
+    import torch
+    if not seqs:
+        raise ValueError("need at least one sequence")
+    H, D = seqs[0].q.shape[1], seqs[0].q.shape[2]
+    arr = (rkv_attn_seq * len(seqs))(*[s.to_c() for s in seqs])
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        workspace = torch.empty(attn_fwd_varlen_workspace_size(len(seqs), H, D), dtype=torch.uint8,
+                                device=seqs[0].q.device)
+    ptr = None
+    if row_stats is not None:
+        rows = sum(int(s.q.shape[0]) for s in seqs)
+        if row_stats.dtype != torch.int32 or not row_stats.is_cuda or not row_stats.is_contiguous() \
+                or row_stats.numel() < rows * H * 4:
+            raise ValueError(f"row_stats must be a contiguous int32 CUDA tensor of >= {rows * H * 4} elements")
+        ptr = row_stats.data_ptr()
+    dbg = rkv_attn_debug(ptr, int(stall), int(timeout_us))
+    _check(_lib.attn_fwd_varlen_debug(arr, len(seqs), H, D, float(softmax_scale), ctypes.byref(rope),
+                                      workspace.data_ptr(), workspace.numel(), ctypes.byref(dbg), _stream(stream)))
+    return workspace
+
+
+def attn_fwd_varlen_noalloc(seqs, rope, softmax_scale=None, stream=None):
+    """attn_fwd_varlen without a caller workspace (the library's fixed scratch)."""
+    if not seqs:
+        raise ValueError("need at least one sequence")
+    H, D = seqs[0].q.shape[1], seqs[0].q.shape[2]
+    arr = (rkv_attn_seq * len(seqs))(*[s.to_c() for s in seqs])
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(_lib.attn_fwd_varlen_noalloc(arr, len(seqs), H, D, float(softmax_scale), ctypes.byref(rope),
+                                        _stream(stream)))
+
+
+def rkv_attn_noalloc_status(stream=None):
+    """Synchronise and raise RkvError if the last no-alloc launch on this GPU timed out."""
+    _check(_lib.rkv_attn_noalloc_status(_stream(stream)))
+
+
 def attn_mask_rows(seqs, H, rope):
     """The mask and key-tile plan attn_fwd_varlen uses for ``seqs``, evaluated
     on the host by the kernel's own code (no GPU needed).  ``seqs``: AttnSeq
@@ -235,6 +305,22 @@ def rkv_ring_status(stream=None):
     _check(_lib.rkv_ring_status(_stream(stream)))
 
 
+def _ring_buffer(t, shape, name):
+    """Check a caller-supplied ring buffer: the kernels write
+    slots * tokens_per_frame * H * D contiguous bf16 values from its start, so
+    anything smaller, strided or on the host is refused here (the C side
+    cannot see a buffer's size)."""
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+        raise ValueError(f"ring {name} must be a bf16 tensor")
+    if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"ring {name} must be a contiguous tensor of shape {tuple(shape)} "
+                         f"(got {tuple(t.shape)}, contiguous={t.is_contiguous()})")
+    if not t.is_cuda:
+        raise ValueError(f"ring {name} must be in CUDA device memory")
+    return t
+
+
 class KVRing:
     """A per-layer ring of frame slots for K and V (device bf16
     [slots][tokens_per_frame][H][D] each) plus its head/count state; the
@@ -245,8 +331,8 @@ class KVRing:
         if not 0 <= pinned < slots:
             raise ValueError(f"pinned ({pinned}) must be in [0, slots={slots})")
         shape = (slots, tokens_per_frame, H, D)
-        self.k = torch.empty(shape, dtype=torch.bfloat16, device=device) if k is None else k
-        self.v = torch.empty(shape, dtype=torch.bfloat16, device=device) if v is None else v
+        self.k = torch.empty(shape, dtype=torch.bfloat16, device=device) if k is None else _ring_buffer(k, shape, "k")
+        self.v = torch.empty(shape, dtype=torch.bfloat16, device=device) if v is None else _ring_buffer(v, shape, "v")
         self.c = rkv_ring(self.k.data_ptr(), self.v.data_ptr(), slots, tokens_per_frame, H, D, pinned, 0, pinned)
 
     @property
@@ -293,6 +379,18 @@ def kvcache_ring_update(ring, k_new, v_new, n_frames=None, stream=None):
     ev = ctypes.c_int32(0)
     _check(_lib.kvcache_ring_update(ctypes.byref(ring.c), k_new.data_ptr(), v_new.data_ptr(), ks, n_frames,
                                     ctypes.byref(ev), _stream(stream)))
+    return ev.value
+
+
+def kvcache_ring_update_debug(ring, k_new, v_new, n_frames=None, stall=RKV_DEBUG_STALL_BULK_LOAD, timeout_us=0,
+                              stream=None):
+    """kvcache_ring_update with stall injection (see rkv.h); returns the
+    number of frames evicted."""
+    ks, n_frames = _ring_insert_args(ring, k_new, v_new, n_frames)
+    ev = ctypes.c_int32(0)
+    dbg = rkv_ring_debug(int(stall), int(timeout_us))
+    _check(_lib.kvcache_ring_update_debug(ctypes.byref(ring.c), k_new.data_ptr(), v_new.data_ptr(), ks, n_frames,
+                                          ctypes.byref(ev), ctypes.byref(dbg), _stream(stream)))
     return ev.value
 
 

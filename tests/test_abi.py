@@ -358,3 +358,43 @@ def test_python_binding_refuses_non_bf16(rkv):
     x = torch.zeros(4, 2, 128, dtype=torch.float32)
     with pytest.raises(ValueError):
         rkv.rope3d_apply(x, rope=rkv.make_rope(4, 6))
+
+
+def test_kvring_refuses_unfit_caller_buffers(rkv):
+    # the ring kernels write slots*F*H*D contiguous bf16 values from the start
+    # of each buffer, so the binding refuses anything that cannot hold them
+    import torch
+    shape = (3, 24, 2, 128)
+    good = torch.zeros(shape, dtype=torch.bfloat16)
+    bad = [torch.zeros(shape, dtype=torch.float16),                         # wrong dtype
+           torch.zeros((2, 24, 2, 128), dtype=torch.bfloat16),             # too few slots
+           torch.zeros((3 * 24 * 2 * 128 - 8,), dtype=torch.bfloat16),     # too few elements
+           torch.zeros((3, 24, 4, 128), dtype=torch.bfloat16)[:, :, :2],   # strided view
+           good]                                                           # host memory
+    for b in bad:
+        with pytest.raises(ValueError):
+            rkv.KVRing(3, 24, 2, k=b, device="cpu")
+        with pytest.raises(ValueError):
+            rkv.KVRing(3, 24, 2, v=b, device="cpu")
+
+
+def test_debug_entry_points_reject_bad_settings(rkv):
+    lib = rkv.lib()
+    arr = (rkv.rkv_attn_seq * 1)(seq(rkv))
+    r = rope(rkv)
+    ws = fake(0x700000)
+    dbg = rkv.rkv_attn_debug(None, 99, 0)
+    assert lib.attn_fwd_varlen_debug(arr, 1, 2, 128, 0.088, ctypes.byref(r), ws, 256, None, None) == \
+        rkv.RKV_ERR_INVALID_ARG
+    assert lib.attn_fwd_varlen_debug(arr, 1, 2, 128, 0.088, ctypes.byref(r), ws, 256, ctypes.byref(dbg), None) == \
+        rkv.RKV_ERR_INVALID_ARG
+    dbg = rkv.rkv_attn_debug(fake(0x800004), 0, 0)   # misaligned record
+    assert lib.attn_fwd_varlen_debug(arr, 1, 2, 128, 0.088, ctypes.byref(r), ws, 256, ctypes.byref(dbg), None) == \
+        rkv.RKV_ERR_INVALID_ARG
+    ring = rkv.rkv_ring(fake(0x100000), fake(0x200000), 3, 24, 2, 128, 0, 0, 0)
+    rd = rkv.rkv_ring_debug(7, 0)
+    ev = ctypes.c_int32(0)
+    assert lib.kvcache_ring_update_debug(ctypes.byref(ring), fake(0x300000), fake(0x400000), 256, 1,
+                                         ctypes.byref(ev), ctypes.byref(rd), None) == rkv.RKV_ERR_INVALID_ARG
+    assert lib.kvcache_ring_update_debug(ctypes.byref(ring), fake(0x300000), fake(0x400000), 256, 1,
+                                         ctypes.byref(ev), None, None) == rkv.RKV_ERR_INVALID_ARG

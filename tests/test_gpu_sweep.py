@@ -99,3 +99,61 @@ def test_sweep_first_layer_all_steps():
 
 def test_sweep_last_layer_all_steps():
     run_layer(SWEEP.layers - 1, SWEEP.steps)
+
+
+@pytest.mark.slow
+def test_sweep_all_layers():
+    """All 30 layers x 8 steps.  Per step: head, count, evicted frames and the
+    slot map bit-exact; the inserted K frames within one bf16 ulp of the
+    correctly rounded fp64 rotation and the inserted V frames bit-exact (in
+    their slots); every other valid slot unchanged since the previous step;
+    attention on sampled query rows (first/last rows, both sides of every
+    frame boundary, random rows) against the oracle ring.  The oracle side of
+    each layer runs in a worker process (tests/_oracle_pool.py)."""
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    from tests._oracle_pool import sweep_layer, workers
+    sw = SWEEP
+    F, H, D, W = sw.frame_tokens, sw.heads, sw.head_dim, sw.ring_slots
+    rope = rkv.make_rope(sw.grid_h, sw.grid_w)
+    ws = torch.zeros(rkv.attn_fwd_varlen_workspace_size(1, H, D), dtype=torch.uint8, device="cuda")
+    ahead = max(2, workers())
+    futs = {layer: sweep_layer(layer, sw.steps) for layer in range(min(sw.layers, ahead))}
+    for layer in range(sw.layers):
+        if layer + ahead < sw.layers:
+            futs[layer + ahead] = sweep_layer(layer + ahead, sw.steps)
+        ring = rkv.KVRing(W, F, H, D)
+        _, k0, v0 = sw.step_inputs(layer, -1)
+        rkv.kvcache_ring_update_rope(ring, to_dev(k0), to_dev(v0), 0, rope, sw.seed_frames)
+        expect = futs.pop(layer).result()
+        for step, ex in enumerate(expect):
+            q_bits, k_bits, v_bits = sw.step_inputs(layer, step)
+            t_new = sw.first_new_frame(step)
+            before_k, before_v = ring.k.clone(), ring.v.clone()
+            kd, vd = to_dev(k_bits), to_dev(v_bits)
+            ev = rkv.kvcache_ring_update_rope(ring, kd, vd, t_new, rope, sw.insert)
+            rkv.rkv_ring_status()
+            where = f"layer {layer} step {step}"
+            assert ev == ex["evicted"], where
+            assert (ring.head, ring.count) == (ex["head"], ex["count"]), where
+            assert [ring.slot(j) for j in range(W)] == ex["slot_map"], where
+            # the inserted frames are the newest sw.insert logical frames
+            new_slots = [ring.slot(ring.count - sw.insert + i) for i in range(sw.insert)]
+            for i, s in enumerate(new_slots):
+                got_k = to_bits(ring.k[s]).reshape(F, H * D)
+                want_k = ex["k_rot"][i * F:(i + 1) * F].reshape(F, H * D)
+                assert int(bf16_ulp_distance(got_k, want_k).max()) <= 1, (where, s)
+                assert torch.equal(ring.v[s], vd[i * F:(i + 1) * F]), (where, s)
+            for s in ex["valid"]:
+                if s not in new_slots:
+                    assert torch.equal(ring.k[s], before_k[s]) and torch.equal(ring.v[s], before_v[s]), (where, s)
+            Lk = ring.count * F
+            q = to_dev(q_bits)
+            o = torch.empty_like(q)
+            seq = rkv.AttnSeq(q, ring.k.view(W * F, H, D)[:Lk], ring.v.view(W * F, H, D)[:Lk], o, q_t0=t_new,
+                              rope_q=True, rope_k=False)
+            rkv.attn_fwd_varlen([seq], rope, workspace=ws)
+            rkv.rkv_attn_status(ws)
+            torch.cuda.synchronize()
+            assert_attn_close(to_f64(o)[ex["rows"]], ex["attn"], f"{where} Lk {Lk}")
+            del before_k, before_v

@@ -6,9 +6,12 @@ caller workspace.
 
 The call goes straight through the C ABI and its output must match the
 regular workspace entry point within the attention tolerances, on two calls in
-a row (the second call reuses the scratch the first one left behind).  This
-file is collected last on purpose, and it passes both on its own in a fresh
-process and after the rest of the suite.
+a row (the second call reuses the scratch the first one left behind).  Around
+those two calls torch's caching allocator must report the same allocated and
+reserved bytes, and the status word the calls left in the library's scratch
+(read back with rkv_attn_noalloc_status, which allocates nothing either) must
+be RKV_OK.  This file is collected last on purpose, and it passes both on its
+own in a fresh process and after the rest of the suite.
 """
 
 import ctypes
@@ -60,11 +63,19 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     ws = rkv.attn_fwd_varlen(ref, rope, softmax_scale=scale)
     rkv.rkv_attn_status(ws)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for call in range(2):
-        seqs = seqs_with_fresh_outputs()
-        arr = (rkv.rkv_attn_seq * len(seqs))(*[s.to_c() for s in seqs])
-        st = fn(arr, len(seqs), H, D, scale, ctypes.byref(rope), stream)
+    status = rkv.lib().rkv_attn_noalloc_status
+    status.restype = ctypes.c_int
+    status.argtypes = [ctypes.c_void_p]
+    calls = [seqs_with_fresh_outputs() for _ in range(2)]
+    arrs = [(rkv.rkv_attn_seq * len(seqs))(*[s.to_c() for s in seqs]) for seqs in calls]
+    torch.cuda.synchronize()
+    allocated, reserved = torch.cuda.memory_allocated(), torch.cuda.memory_reserved()
+    for call, arr in enumerate(arrs):
+        st = fn(arr, len(calls[call]), H, D, scale, ctypes.byref(rope), stream)
         assert st == rkv.RKV_OK, rkv.rkv_last_error_string()
-        torch.cuda.synchronize()
+        assert status(stream) == rkv.RKV_OK, rkv.rkv_last_error_string()
+    torch.cuda.synchronize()
+    assert (torch.cuda.memory_allocated(), torch.cuda.memory_reserved()) == (allocated, reserved)
+    for call, seqs in enumerate(calls):
         for r, s in zip(ref, seqs):
             assert_attn_close(to_f64(s.o), to_f64(r.o), what=f"no-alloc call {call}")
