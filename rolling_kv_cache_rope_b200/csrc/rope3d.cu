@@ -14,6 +14,13 @@
 // result is small against the inputs (cancellation, ~1e-4 of outputs) it is
 // recomputed with error-free transforms so every output rounds to within one
 // bf16 ulp of the exactly rounded value.
+//
+// Adjacent pairs (rope3d_adj_kernel): every thread keeps one 16-byte chunk
+// position of a row (so its four pairs, their axes and table columns are
+// fixed) and walks down the CTA's rows; the table is chunk-major (cos and sin
+// of 4 consecutive pairs at one position, 16 bytes each), so a chunk reads 32
+// bytes of table, and the exact path is out of line.  Rotate-half pairs
+// (rope3d_half_kernel) keep the per-pair table.
 #include <math.h>
 
 #include <algorithm>
@@ -40,15 +47,21 @@ struct RopeArgs {
   int32_t pt, ph, pw;      // rotary pairs per axis
   double log2_theta[3];    // per axis t, h, w
   FastDiv div_F, div_W, div_cpr, div_cph;
+  // adjacent layout: axis a owns rotary pairs [ax_first[a], + ax_count[a]),
+  // i.e. 16-byte chunks [ax_chunk0[a], + ax_nch[a]); chunk g's first and last
+  // pair lie on axes ch_ax_lo[g] and ch_ax_hi[g]
+  int32_t ax_first[3], ax_count[3], ax_chunk0[3], ax_nch[3];
+  int8_t ch_ax_lo[16], ch_ax_hi[16];
 };
 
-// threads per CTA: the standalone op runs one 1024-thread CTA per SM (each
-// cos/sin table serves more rows); the ring insert, a short launch with a V
-// copy beside it, keeps four 256-thread CTAs per SM (measured faster there)
+// threads per CTA (rotate-half kernel): the standalone op runs one 1024-thread
+// CTA per SM (each cos/sin table serves more rows); the ring insert, a short
+// launch with a V copy beside it, keeps four 256-thread CTAs per SM
 template <bool kRing>
 constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
-constexpr int kRopeMaxEntries = 4096;  // 64 KB of float4 per CTA
+constexpr int kRopeMaxEntries = 4096;  // 64 KB of per-pair entries per CTA (rotate-half)
+constexpr int kAdjMaxEntries = 1024;   // 64 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
 
 struct TabEntry {
   float c_hi, s_hi, c_lo, s_lo;
@@ -90,14 +103,14 @@ __device__ __forceinline__ uint8_t* dst_chunk(const RopeArgs& a, uint8_t* base, 
 
 // Ring mode, second tensor: copy rows [r0, r1) of x2 into the ring unrotated.
 __device__ __forceinline__ void copy_rows_to_ring(const RopeArgs& a, uint32_t r0, uint32_t r1) {
-  constexpr int kRopeThreads = rope_threads<true>();
+  const uint32_t T = blockDim.x;
   const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
-  for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
+  for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += T * kRopeUnroll) {
     uint4 v[kRopeUnroll];
     uint8_t* out[kRopeUnroll];
 #pragma unroll
     for (int u = 0; u < kRopeUnroll; ++u) {
-      const uint32_t ci = base + u * kRopeThreads;
+      const uint32_t ci = base + u * T;
       out[u] = nullptr;
       if (ci < c_end) {
         const uint32_t r = fdiv(ci, a.div_cpr);
@@ -135,13 +148,13 @@ __device__ __forceinline__ void rotate_half_chunks(uint4& A, uint4& B, int32_t p
   B = make_uint4(b4[0], b4[1], b4[2], b4[3]);
 }
 
+// Rotate-half layout (pair j = elements j and j + 64 of a head, i.e. element
+// e of chunk c and of chunk c + 8).
 // kRing = false: rotate rows of x into rows of y (rope3d_apply).
 // kRing = true: blockIdx.y = 0 rotates x (K) into ring slots of y, blockIdx.y
 // = 1 copies x2 (V) into ring slots of y2 (kvcache_ring_update_rope).
-// kHalf: rotate-half layout (pair j = elements j and j + 64 of a head, i.e.
-// element e of chunk c and of chunk c + 8); else adjacent pairs (2j, 2j+1).
-template <bool kRing, bool kHalf>
-__global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const RopeArgs a) {
+template <bool kRing>
+__global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_half_kernel(const RopeArgs a) {
   constexpr int kRopeThreads = rope_threads<kRing>();
   extern __shared__ float4 tab_raw[];
   TabEntry* tab = reinterpret_cast<TabEntry*>(tab_raw);
@@ -199,7 +212,7 @@ __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const Rop
   }
   __syncthreads();
 
-  if (kHalf) {
+  {
     // units of work: chunk pairs (c, c + 8) of a head, 8 per head
     const uint32_t p_begin = r0 * a.cph, p_end = r1 * a.cph;
     for (uint32_t base = p_begin + threadIdx.x; base < p_end; base += kRopeThreads * kRopeUnroll) {
@@ -239,49 +252,175 @@ __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_kernel(const Rop
         *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, ca[u] + 8u)) = vb[u];
       }
     }
+  }
+}
+
+// Adjacent layout: rotate the 4 pairs of one 16-byte chunk (word k holds
+// x0 in its low and x1 in its high half) with the chunk's cos C and sin S,
+// in fp32 on packed f32x2 FMAs; `bad` is set when an output cancelled below
+// 2^-12 of its inputs and needs the exact path.
+__device__ __forceinline__ uint4 rotate4(uint4 v, float4 C, float4 S, bool& bad) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+  bool b = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t p = w[2 * h], q = w[2 * h + 1];
+    const float2 x0 = make_float2(bf16lo_to_f32(p), bf16lo_to_f32(q));
+    const float2 x1 = make_float2(bf16hi_to_f32(p), bf16hi_to_f32(q));
+    const float2 nx1 = make_float2(-x1.x, -x1.y);
+    const float2 c = h ? make_float2(C.z, C.w) : make_float2(C.x, C.y);
+    const float2 s = h ? make_float2(S.z, S.w) : make_float2(S.x, S.y);
+    const float2 y0 = __ffma2_rn(x0, c, __fmul2_rn(nx1, s));   // x0 cos - x1 sin
+    const float2 y1 = __ffma2_rn(x0, s, __fmul2_rn(x1, c));    // x0 sin + x1 cos
+    const float la = fmaxf(fabsf(x0.x), fabsf(x1.x)) * 0x1p-12f;
+    const float lb = fmaxf(fabsf(x0.y), fabsf(x1.y)) * 0x1p-12f;
+    b |= (fabsf(y0.x) < la) | (fabsf(y1.x) < la) | (fabsf(y0.y) < lb) | (fabsf(y1.y) < lb);
+    o[2 * h] = pack_bf16x2(y0.x, y1.x);
+    o[2 * h + 1] = pack_bf16x2(y0.y, y1.y);
+  }
+  bad = b;
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The exact path of rotate4 for a chunk that cancelled: each output redone
+// with its cos/sin as hi + lo and error-free products (the same result
+// rotate_pair gives).  Out of line: the main loop carries none of it.
+__device__ __noinline__ uint4 rotate4_exact(uint4 v, float4 C, float4 S, float4 Cl, float4 Sl) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float c[4] = {C.x, C.y, C.z, C.w}, s[4] = {S.x, S.y, S.z, S.w};
+  const float cl[4] = {Cl.x, Cl.y, Cl.z, Cl.w}, sl[4] = {Sl.x, Sl.y, Sl.z, Sl.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float y0, y1;
+    rotate_pair(bf16lo_to_f32(w[k]), bf16hi_to_f32(w[k]), TabEntry{c[k], s[k], cl[k], sl[k]}, y0, y1);
+    o[k] = pack_bf16x2(y0, y1);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z) {
+  return a == 0 ? x : (a == 1 ? y : z);
+}
+
+// Adjacent layout (pairs 2j, 2j+1).  kRing as rope3d_half_kernel.  Table
+// (shared memory, four float4 arrays of E entries: cos hi, sin hi, cos lo,
+// sin lo): entry (axis a, chunk k of the axis, position index i) at
+// tab_base[a] + k * npos[a] + i holds the 4 pairs of chunk ax_chunk0[a] + k;
+// pairs of that chunk outside axis a hold cos 1, sin 0, so a chunk that
+// straddles two axes takes the product of the two cos and the sum of the two
+// sin (exact: one factor is 1, one term 0).
+template <bool kRing>
+__global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
+  extern __shared__ float4 tab4[];
+  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
+  if (r0 >= a.L) return;
+  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
+  if (kRing && blockIdx.y == 1) {
+    copy_rows_to_ring(a, r0, r1);
     return;
   }
-
-  const uint32_t c_begin = r0 * a.cpr, c_end = r1 * a.cpr;
-  for (uint32_t base = c_begin + threadIdx.x; base < c_end; base += kRopeThreads * kRopeUnroll) {
-    uint4 v[kRopeUnroll];
-    uint32_t row[kRopeUnroll], within[kRopeUnroll];
+  // positions this CTA's rows reach: frames f_lo..f_hi; grid rows
+  // h_lo..h_lo+nh-1; columns w_lo, w_lo+1, ... (mod grid_w), nw of them
+  const uint32_t f_lo = fdiv(r0, a.div_F), f_hi = fdiv(r1 - 1, a.div_F);
+  const int32_t nt = int32_t(f_hi - f_lo) + 1;
+  int32_t h_lo = 0, nh = a.grid_h;
+  if (f_lo == f_hi) {
+    h_lo = int32_t(fdiv(r0 - f_lo * a.F, a.div_W));
+    nh = int32_t(fdiv(r1 - 1 - f_lo * a.F, a.div_W)) - h_lo + 1;
+  }
+  int32_t w_lo = 0, nw = a.grid_w;
+  if (r1 - r0 < uint32_t(a.grid_w)) {
+    w_lo = int32_t(r0 - fdiv(r0, a.div_W) * uint32_t(a.grid_w));
+    nw = int32_t(r1 - r0);
+  }
+  const int32_t npos0 = nt, npos1 = nh, npos2 = nw;
+  const int32_t tb0 = 0, tb1 = a.ax_nch[0] * npos0, tb2 = tb1 + a.ax_nch[1] * npos1;
+  const int32_t E = tb2 + a.ax_nch[2] * npos2;
+  float4* tC = tab4;
+  float4* tS = tab4 + E;
+  float4* tCl = tab4 + 2 * E;
+  float4* tSl = tab4 + 3 * E;
+  for (int32_t e = threadIdx.x; e < E; e += blockDim.x) {
+    const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
+    const int32_t np = pick3i(ax, npos0, npos1, npos2);
+    const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
+    const int32_t k = rel / np, pi = rel - k * np;
+    int32_t pos = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
+    if (ax == 2 && pos >= a.grid_w) pos -= a.grid_w;
+    const int32_t chunk = a.ax_chunk0[ax] + k;
+    float c4[4], s4[4], cl4[4], sl4[4];
 #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const uint32_t ci = base + u * kRopeThreads;
-      if (ci < c_end) {
-        row[u] = fdiv(ci, a.div_cpr);
-        within[u] = ci - row[u] * a.cpr;
-        v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(row[u]) * a.x_stride_bytes + uint64_t(within[u]) * 16u);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const int32_t i = 4 * chunk + q - a.ax_first[ax];
+      double sd = 0.0, cd = 1.0;
+      if (i >= 0 && i < a.ax_count[ax])
+        sincos(double(pos) * exp2(-(double(i) / double(a.ax_count[ax])) * a.log2_theta[ax]), &sd, &cd);
+      c4[q] = __double2float_rn(cd);
+      s4[q] = __double2float_rn(sd);
+      cl4[q] = __double2float_rn(cd - double(c4[q]));
+      sl4[q] = __double2float_rn(sd - double(s4[q]));
     }
+    tC[e] = make_float4(c4[0], c4[1], c4[2], c4[3]);
+    tS[e] = make_float4(s4[0], s4[1], s4[2], s4[3]);
+    tCl[e] = make_float4(cl4[0], cl4[1], cl4[2], cl4[3]);
+    tSl[e] = make_float4(sl4[0], sl4[1], sl4[2], sl4[3]);
+  }
+  __syncthreads();
+
+  // thread -> (chunk position c of a row, row phase rsub): `lanes` threads per
+  // row, rpp rows side by side; each thread walks rows r0 + rsub, + rpp, ...
+  const uint32_t T = blockDim.x;
+  const uint32_t lanes = a.cpr < T ? a.cpr : T;
+  const uint32_t rpp = T / lanes;
+  const uint32_t rsub = threadIdx.x / lanes;
+  if (rsub >= rpp) return;
+  for (uint32_t c = threadIdx.x - rsub * lanes; c < a.cpr; c += lanes) {
+    const int32_t g = int32_t(c & 15u);
+    const int alo = a.ch_ax_lo[g], ahi = a.ch_ax_hi[g];
+    const int32_t eb_lo = pick3i(alo, tb0, tb1, tb2) + (g - a.ax_chunk0[alo]) * pick3i(alo, npos0, npos1, npos2);
+    const int32_t eb_hi = pick3i(ahi, tb0, tb1, tb2) + (g - a.ax_chunk0[ahi]) * pick3i(ahi, npos0, npos1, npos2);
+    for (uint32_t rb = r0 + rsub; rb < r1; rb += rpp * kRopeUnroll) {
+      uint4 v[kRopeUnroll];
 #pragma unroll
-    for (int u = 0; u < kRopeUnroll; ++u) {
-      const uint32_t ci = base + u * kRopeThreads;
-      if (ci >= c_end) continue;
-      const uint32_t r = row[u];
-      const uint32_t f = fdiv(r, a.div_F);
-      const uint32_t in_f = r - f * a.F;
-      const uint32_t hh = fdiv(in_f, a.div_W);
-      const uint32_t ww = in_f - hh * uint32_t(a.grid_w);
-      int32_t wi_off = int32_t(ww) - w_lo;
-      if (wi_off < 0) wi_off += a.grid_w;
-      const int32_t ti = int32_t(f - f_lo) * a.pt;
-      const int32_t hi = base_h + (int32_t(hh) - h_lo) * a.ph - a.pt;
-      const int32_t wi = base_w + wi_off * a.pw - a.pt - a.ph;
-      const int32_t p0 = int32_t(within[u] & 15u) * 4;   // first rotary pair of this chunk
-      uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int32_t p = p0 + k;
-        const int32_t idx = p < a.pt ? ti + p : (p < a.pt + a.ph ? hi + p : wi + p);
-        const TabEntry e = tab[idx];
-        float y0, y1;
-        rotate_pair(bf16lo_to_f32(w4[k]), bf16hi_to_f32(w4[k]), e, y0, y1);
-        w4[k] = pack_bf16x2(y0, y1);
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        const uint32_t r = rb + u * rpp;
+        if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c) * 16u);
       }
-      *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, within[u])) =
-          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+#pragma unroll
+      for (int u = 0; u < kRopeUnroll; ++u) {
+        const uint32_t r = rb + u * rpp;
+        if (r >= r1) continue;
+        const uint32_t f = fdiv(r, a.div_F);
+        const uint32_t in_f = r - f * a.F;
+        const uint32_t hh = fdiv(in_f, a.div_W);
+        const uint32_t ww = in_f - hh * uint32_t(a.grid_w);
+        int32_t wi = int32_t(ww) - w_lo;
+        if (wi < 0) wi += a.grid_w;
+        const int32_t ti = int32_t(f - f_lo), hi = int32_t(hh) - h_lo;
+        const int32_t e_lo = eb_lo + pick3i(alo, ti, hi, wi);
+        float4 C = tC[e_lo], S = tS[e_lo];
+        int32_t e_hi = -1;
+        if (alo != ahi) {
+          e_hi = eb_hi + pick3i(ahi, ti, hi, wi);
+          const float4 C2 = tC[e_hi], S2 = tS[e_hi];
+          C = make_float4(C.x * C2.x, C.y * C2.y, C.z * C2.z, C.w * C2.w);
+          S = make_float4(S.x + S2.x, S.y + S2.y, S.z + S2.z, S.w + S2.w);
+        }
+        bool bad;
+        uint4 out = rotate4(v[u], C, S, bad);
+        if (bad) {
+          float4 Cl = tCl[e_lo], Sl = tSl[e_lo];
+          if (e_hi >= 0) {
+            const float4 Cl2 = tCl[e_hi], Sl2 = tSl[e_hi];
+            Cl = make_float4(Cl.x + Cl2.x, Cl.y + Cl2.y, Cl.z + Cl2.z, Cl.w + Cl2.w);
+            Sl = make_float4(Sl.x + Sl2.x, Sl.y + Sl2.y, Sl.z + Sl2.z, Sl.w + Sl2.w);
+          }
+          out = rotate4_exact(v[u], C, S, Cl, Sl);
+        }
+        *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, c)) = out;
+      }
     }
   }
 }
@@ -311,11 +450,8 @@ rkv_status check_rope(const rkv_rope3d* rope, int32_t D) {
   return RKV_OK;
 }
 
-// Fill the rotation part of RopeArgs, pick rows per CTA under the table
-// budget and launch (ring mode: two CTA rows, K rotated and V copied).
-template <bool kRing, bool kHalf>
-static rkv_status launch_rope_shape(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
-                              cudaStream_t stream) {
+// Fill the rotation part of RopeArgs shared by both layouts.
+static void fill_rope_args(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope) {
   a.L = uint32_t(L);
   a.cpr = uint32_t(H) * 16u;
   a.F = uint32_t(rope->grid_h) * uint32_t(rope->grid_w);
@@ -333,6 +469,26 @@ static rkv_status launch_rope_shape(RopeArgs& a, int64_t L, int32_t H, int32_t t
   a.div_F = make_fastdiv(a.F);
   a.div_W = make_fastdiv(uint32_t(rope->grid_w));
   a.div_cpr = make_fastdiv(a.cpr);
+  const int32_t pairs[3] = {rope->pairs_t, rope->pairs_h, rope->pairs_w};
+  int32_t first = 0;
+  for (int ax = 0; ax < 3; ++ax) {
+    a.ax_first[ax] = first;
+    a.ax_count[ax] = pairs[ax];
+    a.ax_chunk0[ax] = first / 4;
+    a.ax_nch[ax] = (first + pairs[ax] - 1) / 4 - first / 4 + 1;
+    first += pairs[ax];
+  }
+  auto axis_of_pair = [&](int pr) { return pr < a.ax_first[1] ? 0 : (pr < a.ax_first[2] ? 1 : 2); };
+  for (int g = 0; g < 16; ++g) {
+    a.ch_ax_lo[g] = int8_t(axis_of_pair(4 * g));
+    a.ch_ax_hi[g] = int8_t(axis_of_pair(4 * g + 3));
+  }
+}
+
+// Rotate-half layout: rows per CTA under the per-pair table budget, launch
+// (ring mode: two CTA rows, K rotated and V copied).
+template <bool kRing>
+static rkv_status launch_rope_half(RopeArgs& a, int64_t L, cudaStream_t stream) {
   const int64_t target_ctas = int64_t(sm_count()) * (kRing ? 4 : 1);
   int64_t rpc = (L + target_ctas - 1) / target_ctas;
   if (rpc < 1) rpc = 1;
@@ -348,20 +504,52 @@ static rkv_status launch_rope_shape(RopeArgs& a, int64_t L, int32_t H, int32_t t
   const size_t smem = size_t(entries(rpc)) * sizeof(TabEntry);
   // set on every launch: the attribute belongs to the current device, and a
   // process may launch on several
-  cudaError_t e = cudaFuncSetAttribute(rope3d_kernel<kRing, kHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(rope3d_half_kernel<kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kRopeMaxEntries * int(sizeof(TabEntry)));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_kernel)");
-  rope3d_kernel<kRing, kHalf><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_half_kernel)");
+  rope3d_half_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), rope_threads<kRing>(), smem, stream>>>(a);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "rope3d_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "rope3d_half_kernel launch");
+  return RKV_OK;
+}
+
+// Adjacent layout: a block is `lanes` threads per row (one per 16-byte chunk,
+// at most 1024) times the rows side by side that fit in 1024 threads (the
+// standalone op, one CTA per SM) or in 256 threads (the ring insert, four
+// CTAs per SM beside the V copy); rows per CTA under the table budget.
+template <bool kRing>
+static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
+  const int64_t lanes = std::min<int64_t>(a.cpr, 1024);
+  const int64_t cap = kRing ? 256 : 1024;
+  const int64_t threads = lanes * std::max<int64_t>(1, cap / lanes);
+  const int64_t target_ctas = int64_t(sm_count()) * (kRing ? 4 : 1);
+  int64_t rpc = (L + target_ctas - 1) / target_ctas;
+  if (rpc < 1) rpc = 1;
+  // upper bound of the chunk entries a CTA of `rows` rows builds (see the kernel)
+  auto entries = [&](int64_t rows) {
+    const int64_t nt = rows / a.F + 2;
+    return int64_t(a.ax_nch[0]) * nt + int64_t(a.ax_nch[1]) * a.grid_h +
+           int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows);
+  };
+  if (entries(1) > kAdjMaxEntries) return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
+  while (rpc > 1 && entries(rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
+  a.rows_per_cta = uint32_t(rpc);
+  const int64_t grid = (L + rpc - 1) / rpc;
+  const size_t smem = size_t(entries(rpc)) * 4 * sizeof(float4);
+  cudaError_t e = cudaFuncSetAttribute(rope3d_adj_kernel<kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kAdjMaxEntries * 4 * int(sizeof(float4)));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_adj_kernel)");
+  rope3d_adj_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), uint32_t(threads), smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rope3d_adj_kernel launch");
   return RKV_OK;
 }
 
 template <bool kRing>
 static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
                               cudaStream_t stream) {
-  return rope->layout == RKV_ROPE_HALF ? launch_rope_shape<kRing, true>(a, L, H, t0, rope, stream)
-                                       : launch_rope_shape<kRing, false>(a, L, H, t0, rope, stream);
+  fill_rope_args(a, L, H, t0, rope);
+  return rope->layout == RKV_ROPE_HALF ? launch_rope_half<kRing>(a, L, stream) : launch_rope_adj<kRing>(a, L, stream);
 }
 
 }  // namespace rkv
