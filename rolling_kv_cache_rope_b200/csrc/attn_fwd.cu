@@ -200,10 +200,21 @@ __device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t b, uint32_t par
 // After the CTA stopped: wait (bounded, without looking at the stop flag) for
 // a TMA load this thread issued to land, so no copy still writes this CTA's
 // shared memory when it exits.
-__device__ __forceinline__ void drain_phase(const Ctx& c, uint32_t b, uint32_t parity) {
+__device__ __forceinline__ void drain_phase(uint32_t b, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = ptx::globaltimer_ns();
   while (!ptx::mbar_try_wait(b, parity))
-    if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) return;
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return;
+}
+
+// The last `stages` loads issued into a ring of `stages` full barriers
+// starting at `bar0` (iterations [it - stages, it)), plus, when q_phases > 0,
+// the last load on barrier `qbar`: wait for each (bounded).  Out of line so
+// the producers' main loops keep their register allocation.
+__device__ __noinline__ void drain_loads(uint32_t bar0, uint32_t it, uint32_t stages, uint32_t qbar,
+                                         uint32_t q_phases, uint64_t limit_ns) {
+  if (q_phases > 0) drain_phase(qbar, (q_phases - 1) & 1u, limit_ns);
+  for (uint32_t i = it > stages ? it - stages : 0u; i < it; ++i)
+    drain_phase(bar0 + 8u * (i % stages), (i / stages) & 1u, limit_ns);
 }
 
 // Debug launches: an index check; a failed one records RKV_ERR_DEVICE_CHECK
@@ -622,8 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t tO = tmem_base + lane_off + col_o(wg);
     const uint32_t pfull = lbar(B_PFULL + wg), ofree = lbar(B_OFREE + wg);
     const float scale_log2 = p.scale_log2;
-    uint32_t g = 0;
-    for (int u = cluster; u < p.total_units; u += n_clusters) {
+    uint32_t g = 0, items = 0;
+    for (int u = cluster; u < p.total_units; u += n_clusters, ++items) {
       const Unit un = decode_unit(p, u);
       const SeqDev& s = p.seq[un.si];
       const int qrow = un.qb * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
@@ -642,18 +653,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // partial tile for some row of the warp: hide keys at or past each
         // row's limit (the keys of a row's mask are a prefix)
         const bool masked = __any_sync(0xffffffffu, lim < kBN);
-        if (masked) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
-        }
-        if constexpr (kDebug) row_stats_tile(sr, uint32_t(kbase), rs);
         const float m_old = m;
         float m_new, tile_sum;
         bool need;
         if (j > un.kt0 && !masked) {
+          if constexpr (kDebug) row_stats_tile(sr, uint32_t(kbase), rs);
           // speculative: exponentials against the running max while the
           // tile max is found; redone (rarely) when the max has to move
           float mx;
@@ -665,6 +669,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tile_sum = exp_store_tile(sr, tS, scale_log2, m);
           }
         } else {
+          if (masked) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (ch * 32 + i >= lim) sr[ch][i] = 0xFF800000u;   // -inf
+          }
+          if constexpr (kDebug) row_stats_tile(sr, uint32_t(kbase), rs);
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
@@ -679,10 +691,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           tile_sum = exp_store_tile(sr, tS, scale_log2, m_use);
         }
         if (j > un.kt0 && __any_sync(0xffffffffu, need)) {
-          // O holds tiles 0..j-1 scaled to the old max: wait for the last PV,
-          // then rescale in TMEM (PV(j) is not issued before P_FULL below)
-          if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 2)) goto done;
-          ptx::tc_fence_after();
+          // O holds tiles 0..j-1 scaled to the old max; S(j) was committed
+          // after PV(j-1), so O is complete; rescale in TMEM (PV(j) is not
+          // issued before P_FULL below)
           const float f = need ? ptx::ex2_approx(m_old - m_new) : 1.0f;
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
@@ -705,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (lane == 0 && !skip) ptx::mbar_arrive_cluster(pfull);
       }
       // epilogue: O / l -> bf16 -> global (row-major [Lq][H][128])
-      if (!wait_warp(c, bar(c, B_ODONE + wg), (g - 1) & 1u, 3)) goto done;
+      if (!wait_warp(c, bar(c, B_ODONE + wg), items & 1u, 3)) goto done;
       ptx::tc_fence_after();
       {
         const float inv = l > 0.f ? 1.0f / l : 0.f;
@@ -860,12 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         if (!ok) { ++ul; break; }
       }
-      if (!ok) {
-        // stopped early: let this thread's last Q load and K loads land
-        if (ul > 0) drain_phase(c, bar(c, B_QFULL), (ul - 1) & 1u);
-        for (uint32_t i = it > uint32_t(kStages) ? it - kStages : 0u; i < it; ++i)
-          drain_phase(c, bar(c, B_KFULL + i % kStages), (i / kStages) & 1u);
-      }
+      // stopped early: let this thread's last Q load and K loads land
+      if (!ok) drain_loads(bar(c, B_KFULL), it, kStages, bar(c, B_QFULL), ul, p.timeout_ns);
     } else if (warp == 14 && lane == 0) {
       // ===================== TMA producer: this CTA's V column half =====================
       for (int i = 0; i < p.n_seqs; ++i) ptx::tma_prefetch_desc(&p.seq[i].tv);
@@ -881,11 +888,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::tma_load_3d(sV + st * kVStageBytes, &s.tv, bar(c, B_VFULL + st), int(rank) * 64, un.head, j * kBN);
         }
       }
-      if (!ok) {
-        // stopped early: let this thread's last V loads land
-        for (uint32_t i = it > uint32_t(kStages) ? it - kStages : 0u; i < it; ++i)
-          drain_phase(c, bar(c, B_VFULL + i % kStages), (i / kStages) & 1u);
-      }
+      // stopped early: let this thread's last V loads land
+      if (!ok) drain_loads(bar(c, B_VFULL), it, kStages, 0u, 0u, p.timeout_ns);
     } else if (warp == 15 && lane == 0) {
       // ===================== V landed -> tell the leader =====================
       uint32_t it = 0;
@@ -936,7 +940,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
               for (int kk = 0; kk < 8; ++kk)
                 ptx::mma2_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)),
                              id_pv, (j > 1 || kk > 0) ? 1u : 0u);
-              ptx::mma2_commit_mc(bar(c, B_ODONE + b), kBoth);
               // S_b(j) = Q_b K(j)^T: Q rows from each CTA, keys split 64 + 64
               const uint64_t dq = b ? dq1 : dq0;
 #pragma unroll
