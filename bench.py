@@ -653,18 +653,29 @@ def profile_case(args):
     return 0
 
 
+ATTN_SOURCES = ("rolling_kv_cache_rope_b200/csrc/attn_fwd.cu", "rolling_kv_cache_rope_b200/csrc/sm100_ptx.cuh",
+                "rolling_kv_cache_rope_b200/csrc/common.cuh")
+
+
+def attn_source_sha256():
+    """sha256 over the attention kernel's source files, in ATTN_SOURCES order."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def load_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, or None
-    when the attention source has changed since that capture."""
-    import hashlib
+    when the attention kernel's sources have changed since that capture."""
     p = os.path.join(ROOT, "profiles", "attn_fwd_kernel_denoise_23400x32760.md")
-    src = os.path.join(ROOT, "rolling_kv_cache_rope_b200", "csrc", "attn_fwd.cu")
     try:
         with open(p) as f:
             kv = dict(line.split(":", 1) for line in f.read().splitlines()
                       if line.startswith(("source_sha256:", "dram_bytes_per_launch:")))
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = attn_source_sha256()
     except (OSError, ValueError):
         return None
     if kv.get("source_sha256", "").strip() != sha:

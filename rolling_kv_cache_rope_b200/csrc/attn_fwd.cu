@@ -184,11 +184,24 @@ __device__ __forceinline__ bool wait_phase(const Ctx& c, uint32_t b, uint32_t pa
   }
 }
 
-// The same for a barrier that the peer CTA also arrives on.  The handoffs
-// through such barriers carry TMEM or async-proxy shared-memory data, ordered
-// by tcgen05 / proxy fences, so the wait keeps the default (CTA) scope.
+// The MMA issuer's wait (on barriers the peer CTA also arrives on): one
+// thread, on the critical path of every key tile, so it polls without the
+// suspend hint (measured a few percent faster than sleeping there).  The
+// handoffs through these barriers carry TMEM or async-proxy shared-memory
+// data, ordered by tcgen05 / proxy fences, so the wait keeps the default
+// (CTA) scope.  Bounded like wait_phase.
 __device__ __forceinline__ bool wait_phase_cluster(const Ctx& c, uint32_t b, uint32_t parity, int where) {
-  return wait_phase(c, b, parity, where);
+  if (ptx::mbar_try_wait(b, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(b, parity)) return true;
+    if (*c.abort) return false;
+    if (ptx::globaltimer_ns() - t0 > c.p->timeout_ns) {
+      *c.abort = 1;
+      atomicCAS(c.p->status, 0, int(RKV_ERR_TIMEOUT) | (where << 8));
+      return false;
+    }
+  }
 }
 
 // Warp-uniform variant for roles whose 32 lanes continue together.
@@ -923,8 +936,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int nk = un.kt1 - un.kt0;   // tiles of this item; j counts them from 0
         for (int j = 0; j < nk; ++j, ++it, ++g) {
           const uint32_t st = it % kStages, n = it / kStages;
-          if (!wait_phase_cluster(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
           const uint64_t dk = desc_kmajor(sK + st * kKStageBytes);
+          // K(j) is waited for only where S(j) needs it: PV of tile j - 1
+          // below does not, so it is not held up by K(j)'s rotation
+          if (j == 0 && !wait_phase_cluster(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
           if (j > 0) {
             const uint32_t sp = (it - 1) % kStages, np = (it - 1) / kStages;
             if (!wait_phase_cluster(c, bar(c, B_VREADY + sp), np & 1u, 11)) { ok = false; break; }
@@ -940,6 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
               for (int kk = 0; kk < 8; ++kk)
                 ptx::mma2_ts(tmem_base + col_o(b), tmem_base + col_s(b) + 8 * kk, dv + uint64_t(kk * (2048 >> 4)),
                              id_pv, (j > 1 || kk > 0) ? 1u : 0u);
+              if (b == 0 && !wait_phase_cluster(c, bar(c, B_KREADY + st), n & 1u, 10)) { ok = false; break; }
               // S_b(j) = Q_b K(j)^T: Q rows from each CTA, keys split 64 + 64
               const uint64_t dq = b ? dq1 : dq0;
 #pragma unroll
