@@ -54,8 +54,11 @@
 #include <string.h>
 
 #include <algorithm>
+#include <functional>
 #include <mutex>
+#include <queue>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -79,6 +82,8 @@ constexpr int kKStageBytes = kKRows * kHD * 2; // 16 KB: 64 rows x 128 cols
 constexpr int kKHalfBytes = kKStageBytes / 2;  // 64 rows x 64 cols
 constexpr int kVStageBytes = kBN * 64 * 2;     // 16 KB: 128 rows x 64 cols
 constexpr int kThreads = 16 * 32;
+constexpr int kMaxClusters = 128;    // CTA pairs a launch can have (74 on a B200)
+constexpr int kMaxSched = 4096;      // work items a host-built schedule can list
 constexpr int kTabEntryBytes = 32;   // cos and sin of 4 consecutive rotary pairs
 constexpr int kMaxTabEntries = 768;  // 24 KB of shared memory (cos array, then sin array)
 constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growth
@@ -144,6 +149,13 @@ struct Params {
   // [4] int32 or null, and the handoff to skip (RKV_DEBUG_STALL_*)
   int32_t* row_stats;
   uint32_t stall;
+  // work-item schedule: 0 = round-robin (cluster c takes items c, c + C, ...);
+  // 1 = cluster c takes items sched[sched_off[c] .. sched_off[c + 1]) in that
+  // order (a longest-first assignment built on the host when items differ in
+  // cost, e.g. frame-block-masked sequences)
+  int32_t use_sched;
+  uint16_t sched_off[kMaxClusters + 1];
+  uint16_t sched[kMaxSched];
 };
 
 // barrier indices.  The first group is used in every CTA; the second only in
@@ -258,6 +270,15 @@ __device__ __forceinline__ void row_stats_tile(const uint32_t (&sr)[4][32], uint
       st.top = vis ? idx + 1u : st.top;
     }
   st.tiles += 1u;
+}
+
+// Work items of CTA pair `cluster` of `n_clusters`: how many, and the k-th.
+__device__ __forceinline__ int items_of(const Params& p, int cluster, int n_clusters) {
+  if (p.use_sched) return int(p.sched_off[cluster + 1]) - int(p.sched_off[cluster]);
+  return cluster < p.total_units ? (p.total_units - cluster + n_clusters - 1) / n_clusters : 0;
+}
+__device__ __forceinline__ int item_at(const Params& p, int cluster, int n_clusters, int k) {
+  return p.use_sched ? int(p.sched[p.sched_off[cluster] + k]) : cluster + k * n_clusters;
 }
 
 struct Unit {
@@ -569,6 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t rank = ptx::cluster_ctarank();   // 0 = leader of the pair
   const int cluster = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
+  const int n_items = items_of(p, cluster, n_clusters);   // work items of this CTA pair
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8);
   int* abort_flag = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 4);
@@ -647,8 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t pfull = lbar(B_PFULL + wg), ofree = lbar(B_OFREE + wg);
     const float scale_log2 = p.scale_log2;
     uint32_t g = 0, items = 0;
-    for (int u = cluster; u < p.total_units; u += n_clusters, ++items) {
-      const Unit un = decode_unit(p, u);
+    for (int k = 0; k < n_items; ++k, ++items) {
+      const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
       const SeqDev& s = p.seq[un.si];
       const int qrow = un.qb * kUnitRows + int(rank) * kCtaRows + wg * kBM + 32 * (warp & 3) + lane;
       const int64_t my_limit = row_kv_limit(s, p, qrow < s.Lq ? qrow : s.Lq - 1);
@@ -792,8 +814,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int rt = tid - 256;
     const uint32_t qready = lbar(B_QREADY);
     uint32_t it = 0, ul = 0;
-    for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
-      const Unit un = decode_unit(p, u);
+    for (int k = 0; k < n_items; ++k, ++ul) {
+      const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
       const SeqDev& s = p.seq[un.si];
       // Every RoPE warp reaches the named barrier below, whether its own wait
       // succeeded or not, and the barrier's AND takes the stop decision for
@@ -861,8 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       uint32_t it = 0, ul = 0;
       bool ok = true;
-      for (int u = cluster; u < p.total_units; u += n_clusters, ++ul) {
-        const Unit un = decode_unit(p, u);
+      for (int k = 0; k < n_items; ++k, ++ul) {
+        const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
         const SeqDev& s = p.seq[un.si];
         if (!wait_phase(c, bar(c, B_QFREE), (ul & 1u) ^ 1u, 6)) { ok = false; break; }
         if constexpr (kDebug) {
@@ -891,8 +913,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int i = 0; i < p.n_seqs; ++i) ptx::tma_prefetch_desc(&p.seq[i].tv);
       uint32_t it = 0;
       bool ok = true;
-      for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
-        const Unit un = decode_unit(p, u);
+      for (int k = 0; ok && k < n_items; ++k) {
+        const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
         const SeqDev& s = p.seq[un.si];
         for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
@@ -907,8 +929,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       // ===================== V landed -> tell the leader =====================
       uint32_t it = 0;
       bool ok = true;
-      for (int u = cluster; ok && u < p.total_units; u += n_clusters) {
-        const Unit un = decode_unit(p, u);
+      for (int k = 0; ok && k < n_items; ++k) {
+        const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
         for (int j = un.kt0; j < un.kt1; ++j, ++it) {
           const uint32_t st = it % kStages, n = it / kStages;
           if (!wait_phase(c, bar(c, B_VFULL + st), n & 1u, 17)) { ok = false; break; }
@@ -930,8 +952,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       constexpr uint16_t kBoth = 3;
       uint32_t it = 0, g = 0, ul = 0;
       bool ok = true;
-      for (int u = cluster; ok && u < p.total_units; u += n_clusters, ++ul) {
-        const Unit un = decode_unit(p, u);
+      for (int k = 0; ok && k < n_items; ++k, ++ul) {
+        const Unit un = decode_unit(p, item_at(p, cluster, n_clusters, k));
         if (!wait_phase_cluster(c, bar(c, B_QREADY), ul & 1u, 9)) { ok = false; break; }
         const int nk = un.kt1 - un.kt0;   // tiles of this item; j counts them from 0
         for (int j = 0; j < nk; ++j, ++it, ++g) {
@@ -1149,6 +1171,51 @@ static rkv_status attn_launch_shape(bool default_split, bool half, bool debug, c
 // Units of the last, partly filled wave of the persistent grid that are run as
 // two half-units (split over their key tiles) so the wave finishes in about
 // half the time; 0 when the last wave is more than half full.
+// Cost of a unit in the schedule: its key tiles plus a few tiles' worth of
+// per-unit work (Q load and rotation, epilogue).
+constexpr int kUnitOverheadTiles = 4;
+
+// Longest-first assignment of the units to the CTA pairs when their costs
+// differ: units in decreasing cost, each to the pair with the least work so
+// far (greedy LPT, within a few percent of the optimal makespan here).
+// Fills p.use_sched, p.sched_off, p.sched; returns false (round-robin) when
+// every unit costs the same or the launch is too large for the table.
+static bool build_schedule(Params& p, int64_t units, int max_clusters) {
+  p.use_sched = 0;
+  if (units < 2 || units > kMaxSched) return false;
+  const int C = int(std::min<int64_t>(units, max_clusters));
+  if (C > kMaxClusters) return false;
+  const size_t n = size_t(units);
+  std::vector<int> cost(n);
+  bool same = true;
+  for (int u = 0; u < int(units); ++u) {
+    cost[size_t(u)] = decode_unit(p, u).nkt + kUnitOverheadTiles;
+    same = same && cost[size_t(u)] == cost[0];
+  }
+  if (same) return false;
+  std::vector<int> order(n);
+  for (int u = 0; u < int(units); ++u) order[size_t(u)] = u;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[size_t(a)] > cost[size_t(b)]; });
+  using Load = std::pair<int64_t, int>;   // (work so far, pair)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < C; ++c) heap.push({0, c});
+  std::vector<std::vector<int>> lists(static_cast<size_t>(C));
+  for (int u : order) {
+    Load l = heap.top();
+    heap.pop();
+    lists[size_t(l.second)].push_back(u);
+    heap.push({l.first + cost[size_t(u)], l.second});
+  }
+  int at = 0;
+  for (int c = 0; c < C; ++c) {
+    p.sched_off[c] = uint16_t(at);
+    for (int u : lists[size_t(c)]) p.sched[at++] = uint16_t(u);
+  }
+  p.sched_off[C] = uint16_t(at);
+  p.use_sched = 1;
+  return true;
+}
+
 static int tail_split_units(int64_t units, int clusters) {
   if (clusters < 2 || units <= clusters) return 0;
   const int64_t rest = units % clusters;
@@ -1345,10 +1412,14 @@ static rkv_status attn_launch(const rkv_attn_seq* seqs, int32_t n_seqs, int32_t 
     return st;
   cfg.stream = cs;
 
+  // Units of different cost (frame-block-masked sequences, or sequences of
+  // different lengths in one launch) get a longest-first schedule; units of
+  // one cost keep round-robin with the tail split below.
+  const bool sched = build_schedule(p, units, max_clusters);
   // tail split: the last n_split units run as two half-units each when the
   // workspace can hold their partial results and every such unit has >= 2
   // key tiles
-  int n_split = tail_split_units(units, max_clusters);
+  int n_split = sched ? 0 : tail_split_units(units, max_clusters);
   if (workspace_bytes < kWorkspaceBytes + size_t(2 * n_split) * kPartBytesPerItem) n_split = 0;
   CombineArgs ca;
   memset(&ca, 0, sizeof(ca));

@@ -3,7 +3,10 @@ most half full, its units run as two halves over their key tiles and a second
 kernel merges the halves.  These cases make that happen with small shapes
 (more units than CTA pairs on a B200) and check every output against the fp64
 oracle, and against the same launch with a workspace too small for the split
-(no split), unmasked and frame-block masked."""
+(no split), unmasked and frame-block masked.  The split applies when every
+work unit costs the same; launches whose units differ in cost (most masked
+or mixed-length launches) are scheduled longest-first instead, which the
+masked and varlen cases of the other attention tests cover."""
 
 import math
 
@@ -35,11 +38,12 @@ def run(Lq, Lk, H, grid_h, grid_w, q_t0, block_frames, q_frame_offset, seed, ws_
     return o
 
 
-def check(Lq, Lk, H, grid_h, grid_w, block_frames, seed):
+def check(Lq, Lk, H, grid_h, grid_w, block_frames, seed, q_frame_offset=None):
     need_gpu()
     from rolling_kv_cache_rope_b200 import rkv
     F = grid_h * grid_w
-    q_frame_offset = max(0, Lk // F - Lq // F)   # query frames are the last ones of the context
+    if q_frame_offset is None:
+        q_frame_offset = max(0, Lk // F - Lq // F)   # query frames are the last ones of the context
     q_t0 = q_frame_offset
     full = rkv.attn_fwd_varlen_workspace_size(1, H, D)
     assert full > 256, "workspace has no room for split partial results"
@@ -63,5 +67,9 @@ def test_tail_split_unmasked():
 
 
 def test_tail_split_frame_block_masked():
-    # 128-token frames, blocks of 3 frames: units see 3..30 key frames
-    check(Lq=28 * 128, Lk=30 * 128, H=12, grid_h=8, grid_w=16, block_frames=3, seed=701)
+    # 120-token frames, blocks of 3 frames, query frame 0 = key frame 24: the
+    # first 360 query rows see 27 key frames (3,240 keys, a partial tile),
+    # every later row all 3,600 keys, and every 512-row unit ends on a row
+    # that sees them all, so all 84 units cost the same and the last 10 run
+    # as halves
+    check(Lq=7 * 512, Lk=30 * 120, H=12, grid_h=8, grid_w=15, block_frames=3, seed=701, q_frame_offset=24)

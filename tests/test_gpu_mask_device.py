@@ -127,10 +127,17 @@ def test_three_sequences_one_launch():
 
 @pytest.mark.parametrize("split", [True, False])
 def test_tail_split_masked(split):
-    # 12 heads x 7 blocks of 512 query rows = 84 units on 74 CTA pairs: with
-    # the split the last 10 units run as two halves over their key tiles
-    Lq, Lk = 28 * 128, 30 * 128
-    check([S(Lq, Lk, 3, Lk // 128 - Lq // 128)], 12, 8, 16, split=split)
+    # 12 heads x 7 blocks of 512 query rows = 84 units on 74 CTA pairs, all of
+    # the same cost (each unit's last row sees all 3,600 keys; the first 360
+    # rows see 3,240, a partial tile): with the split the last 10 units run as
+    # two halves over their key tiles, and their records add up
+    check([S(7 * 512, 30 * 120, 3, 24, q_t0=24)], 12, 8, 15, split=split)
+
+
+def test_masked_longest_first_schedule():
+    # units of different cost (128-token frames, query frames 0.. see 3 to 30
+    # key frames): scheduled longest-first over the CTA pairs
+    check([S(28 * 128, 30 * 128, 3, 0)], 12, 8, 16)
 
 
 @pytest.mark.slow
