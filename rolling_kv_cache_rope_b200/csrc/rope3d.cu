@@ -19,8 +19,9 @@
 // position of a row (so its four pairs, their axes and table columns are
 // fixed) and walks down the CTA's rows; the table is chunk-major (cos and sin
 // of 4 consecutive pairs at one position, 16 bytes each), so a chunk reads 32
-// bytes of table, and the exact path is out of line.  Rotate-half pairs
-// (rope3d_half_kernel) keep the per-pair table.
+// bytes of table, and the exact path is out of line.  A chunk whose pairs lie
+// on two or three axes reads per-row entries, so every chunk takes the same
+// path.  Rotate-half pairs (rope3d_half_kernel) keep the per-pair table.
 #include <math.h>
 
 #include <algorithm>
@@ -48,10 +49,12 @@ struct RopeArgs {
   double log2_theta[3];    // per axis t, h, w
   FastDiv div_F, div_W, div_cpr, div_cph;
   // adjacent layout: axis a owns rotary pairs [ax_first[a], + ax_count[a]),
-  // i.e. 16-byte chunks [ax_chunk0[a], + ax_nch[a]); chunk g's first and last
-  // pair lie on axes ch_ax_lo[g] and ch_ax_hi[g]
+  // i.e. 16-byte chunks [ax_chunk0[a], + ax_nch[a]).  Chunk g's four pairs lie
+  // on one axis, ch_axis[g], or on two or three (ch_axis[g] = -1): such a
+  // chunk reads per-row table entries, region ch_multi[g] of n_multi
   int32_t ax_first[3], ax_count[3], ax_chunk0[3], ax_nch[3];
-  int8_t ch_ax_lo[16], ch_ax_hi[16];
+  int8_t ch_axis[16], ch_multi[16];
+  int32_t n_multi;
 };
 
 // threads per CTA (rotate-half kernel): the standalone op runs one 1024-thread
@@ -304,13 +307,40 @@ __device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z
   return a == 0 ? x : (a == 1 ? y : z);
 }
 
+// Table entry of 16-byte chunk `chunk` (rotary pairs 4*chunk .. +3) at
+// positions (p_t, p_h, p_w): cos and sin of each pair's angle rounded to
+// fp32 (hi) and the fp32 rounding of the rest (lo).  Pairs on an axis outside
+// the bit mask `axes` hold cos 1, sin 0.
+__device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_t, int32_t p_h, int32_t p_w, float4& C, float4& S,
+                          float4& Cl, float4& Sl) {
+  float c4[4], s4[4], cl4[4], sl4[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int32_t pr = 4 * chunk + q;
+    const int ax = pr < a.ax_first[1] ? 0 : (pr < a.ax_first[2] ? 1 : 2);
+    const int32_t i = pr - a.ax_first[ax];
+    double sd = 0.0, cd = 1.0;
+    if ((axes >> ax) & 1)
+      sincos(double(pick3i(ax, p_t, p_h, p_w)) * exp2(-(double(i) / double(a.ax_count[ax])) * a.log2_theta[ax]), &sd, &cd);
+    c4[q] = __double2float_rn(cd);
+    s4[q] = __double2float_rn(sd);
+    cl4[q] = __double2float_rn(cd - double(c4[q]));
+    sl4[q] = __double2float_rn(sd - double(s4[q]));
+  }
+  C = make_float4(c4[0], c4[1], c4[2], c4[3]);
+  S = make_float4(s4[0], s4[1], s4[2], s4[3]);
+  Cl = make_float4(cl4[0], cl4[1], cl4[2], cl4[3]);
+  Sl = make_float4(sl4[0], sl4[1], sl4[2], sl4[3]);
+}
+
 // Adjacent layout (pairs 2j, 2j+1).  kRing as rope3d_half_kernel.  Table
 // (shared memory, four float4 arrays of E entries: cos hi, sin hi, cos lo,
-// sin lo): entry (axis a, chunk k of the axis, position index i) at
-// tab_base[a] + k * npos[a] + i holds the 4 pairs of chunk ax_chunk0[a] + k;
-// pairs of that chunk outside axis a hold cos 1, sin 0, so a chunk that
-// straddles two axes takes the product of the two cos and the sum of the two
-// sin (exact: one factor is 1, one term 0).
+// sin lo).  Entry (axis a, chunk k of the axis, position index i) at
+// tab_base[a] + k * npos[a] + i holds the 4 pairs of chunk ax_chunk0[a] + k
+// (pairs of that chunk outside axis a hold cos 1, sin 0); a chunk whose pairs
+// lie on several axes instead reads entry (region m, row r - r0) after those,
+// built for each of the CTA's rows.  So every chunk reads one entry, and the
+// threads of a warp take the same path whatever chunk positions they hold.
 template <bool kRing>
 __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   extern __shared__ float4 tab4[];
@@ -336,36 +366,43 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
     nw = int32_t(r1 - r0);
   }
   const int32_t npos0 = nt, npos1 = nh, npos2 = nw;
+  const int32_t nrows = int32_t(r1 - r0);
   const int32_t tb0 = 0, tb1 = a.ax_nch[0] * npos0, tb2 = tb1 + a.ax_nch[1] * npos1;
-  const int32_t E = tb2 + a.ax_nch[2] * npos2;
+  const int32_t tbm = tb2 + a.ax_nch[2] * npos2;
+  const int32_t E = tbm + a.n_multi * nrows;
   float4* tC = tab4;
   float4* tS = tab4 + E;
   float4* tCl = tab4 + 2 * E;
   float4* tSl = tab4 + 3 * E;
   for (int32_t e = threadIdx.x; e < E; e += blockDim.x) {
-    const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
-    const int32_t np = pick3i(ax, npos0, npos1, npos2);
-    const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
-    const int32_t k = rel / np, pi = rel - k * np;
-    int32_t pos = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
-    if (ax == 2 && pos >= a.grid_w) pos -= a.grid_w;
-    const int32_t chunk = a.ax_chunk0[ax] + k;
-    float c4[4], s4[4], cl4[4], sl4[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int32_t i = 4 * chunk + q - a.ax_first[ax];
-      double sd = 0.0, cd = 1.0;
-      if (i >= 0 && i < a.ax_count[ax])
-        sincos(double(pos) * exp2(-(double(i) / double(a.ax_count[ax])) * a.log2_theta[ax]), &sd, &cd);
-      c4[q] = __double2float_rn(cd);
-      s4[q] = __double2float_rn(sd);
-      cl4[q] = __double2float_rn(cd - double(c4[q]));
-      sl4[q] = __double2float_rn(sd - double(s4[q]));
+    int32_t pos[3], chunk;
+    int axes;
+    if (e < tbm) {
+      const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
+      const int32_t np = pick3i(ax, npos0, npos1, npos2);
+      const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
+      const int32_t k = rel / np, pi = rel - k * np;
+      int32_t ps = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
+      if (ax == 2 && ps >= a.grid_w) ps -= a.grid_w;
+      pos[0] = pos[1] = pos[2] = ps;
+      chunk = a.ax_chunk0[ax] + k;
+      axes = 1 << ax;
+    } else {
+      // multi-axis chunk: the m-th such chunk position at row r
+      const int32_t m = (e - tbm) / nrows;
+      const uint32_t r = r0 + uint32_t(e - tbm - m * nrows);
+      const uint32_t f = fdiv(r, a.div_F);
+      const uint32_t in_f = r - f * a.F;
+      const uint32_t hh = fdiv(in_f, a.div_W);
+      pos[0] = a.t0 + int32_t(f);
+      pos[1] = int32_t(hh);
+      pos[2] = int32_t(in_f - hh * uint32_t(a.grid_w));
+      chunk = 0;
+      for (int g = 0, seen = 0; g < 16; ++g)
+        if (a.ch_axis[g] < 0 && seen++ == m) chunk = g;
+      axes = 7;
     }
-    tC[e] = make_float4(c4[0], c4[1], c4[2], c4[3]);
-    tS[e] = make_float4(s4[0], s4[1], s4[2], s4[3]);
-    tCl[e] = make_float4(cl4[0], cl4[1], cl4[2], cl4[3]);
-    tSl[e] = make_float4(sl4[0], sl4[1], sl4[2], sl4[3]);
+    adj_entry(a, chunk, axes, pos[0], pos[1], pos[2], tC[e], tS[e], tCl[e], tSl[e]);
   }
   __syncthreads();
 
@@ -377,10 +414,19 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   const uint32_t rsub = threadIdx.x / lanes;
   if (rsub >= rpp) return;
   for (uint32_t c = threadIdx.x - rsub * lanes; c < a.cpr; c += lanes) {
+    // entry of row r: eb + ti*mt + hi*mh + wi*mw + r*mr, one term non-zero
     const int32_t g = int32_t(c & 15u);
-    const int alo = a.ch_ax_lo[g], ahi = a.ch_ax_hi[g];
-    const int32_t eb_lo = pick3i(alo, tb0, tb1, tb2) + (g - a.ax_chunk0[alo]) * pick3i(alo, npos0, npos1, npos2);
-    const int32_t eb_hi = pick3i(ahi, tb0, tb1, tb2) + (g - a.ax_chunk0[ahi]) * pick3i(ahi, npos0, npos1, npos2);
+    const int ax = a.ch_axis[g];
+    int32_t eb, mt = 0, mh = 0, mw = 0, mr = 0;
+    if (ax >= 0) {
+      eb = pick3i(ax, tb0, tb1, tb2) + (g - a.ax_chunk0[ax]) * pick3i(ax, npos0, npos1, npos2);
+      mt = ax == 0;
+      mh = ax == 1;
+      mw = ax == 2;
+    } else {
+      eb = tbm + int32_t(a.ch_multi[g]) * nrows - int32_t(r0);
+      mr = 1;
+    }
     for (uint32_t rb = r0 + rsub; rb < r1; rb += rpp * kRopeUnroll) {
       uint4 v[kRopeUnroll];
 #pragma unroll
@@ -399,26 +445,11 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
         int32_t wi = int32_t(ww) - w_lo;
         if (wi < 0) wi += a.grid_w;
         const int32_t ti = int32_t(f - f_lo), hi = int32_t(hh) - h_lo;
-        const int32_t e_lo = eb_lo + pick3i(alo, ti, hi, wi);
-        float4 C = tC[e_lo], S = tS[e_lo];
-        int32_t e_hi = -1;
-        if (alo != ahi) {
-          e_hi = eb_hi + pick3i(ahi, ti, hi, wi);
-          const float4 C2 = tC[e_hi], S2 = tS[e_hi];
-          C = make_float4(C.x * C2.x, C.y * C2.y, C.z * C2.z, C.w * C2.w);
-          S = make_float4(S.x + S2.x, S.y + S2.y, S.z + S2.z, S.w + S2.w);
-        }
+        const int32_t e = eb + ti * mt + hi * mh + wi * mw + int32_t(r) * mr;
+        const float4 C = tC[e], S = tS[e];
         bool bad;
         uint4 out = rotate4(v[u], C, S, bad);
-        if (bad) {
-          float4 Cl = tCl[e_lo], Sl = tSl[e_lo];
-          if (e_hi >= 0) {
-            const float4 Cl2 = tCl[e_hi], Sl2 = tSl[e_hi];
-            Cl = make_float4(Cl.x + Cl2.x, Cl.y + Cl2.y, Cl.z + Cl2.z, Cl.w + Cl2.w);
-            Sl = make_float4(Sl.x + Sl2.x, Sl.y + Sl2.y, Sl.z + Sl2.z, Sl.w + Sl2.w);
-          }
-          out = rotate4_exact(v[u], C, S, Cl, Sl);
-        }
+        if (bad) out = rotate4_exact(v[u], C, S, tCl[e], tSl[e]);
         *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, c)) = out;
       }
     }
@@ -479,9 +510,11 @@ static void fill_rope_args(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const 
     first += pairs[ax];
   }
   auto axis_of_pair = [&](int pr) { return pr < a.ax_first[1] ? 0 : (pr < a.ax_first[2] ? 1 : 2); };
+  a.n_multi = 0;
   for (int g = 0; g < 16; ++g) {
-    a.ch_ax_lo[g] = int8_t(axis_of_pair(4 * g));
-    a.ch_ax_hi[g] = int8_t(axis_of_pair(4 * g + 3));
+    const int lo = axis_of_pair(4 * g), hi = axis_of_pair(4 * g + 3);
+    a.ch_axis[g] = int8_t(lo == hi ? lo : -1);
+    a.ch_multi[g] = int8_t(lo == hi ? -1 : a.n_multi++);
   }
 }
 
@@ -529,7 +562,7 @@ static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
   auto entries = [&](int64_t rows) {
     const int64_t nt = rows / a.F + 2;
     return int64_t(a.ax_nch[0]) * nt + int64_t(a.ax_nch[1]) * a.grid_h +
-           int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows);
+           int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows) + int64_t(a.n_multi) * rows;
   };
   if (entries(1) > kAdjMaxEntries) return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
   while (rpc > 1 && entries(rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;

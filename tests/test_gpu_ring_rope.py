@@ -20,13 +20,13 @@ pytestmark = pytest.mark.gpu
 SENTINEL = 0x7FC1
 
 
-def run_ring_rope(slots, grid_h, grid_w, H, inserts, seed, stride_mult=1, t_start=0):
+def run_ring_rope(slots, grid_h, grid_w, H, inserts, seed, stride_mult=1, t_start=0, pairs=(22, 21, 21)):
     need_gpu()
     from rolling_kv_cache_rope_b200 import rkv
     D = 128
     F = grid_h * grid_w
     frame_elems = F * H * D
-    rope = rkv.make_rope(grid_h, grid_w)
+    rope = rkv.make_rope(grid_h, grid_w, pairs)
     kbuf = torch.full(((slots + 2) * frame_elems,), SENTINEL, dtype=torch.int16, device="cuda")
     vbuf = torch.full(((slots + 2) * frame_elems,), SENTINEL, dtype=torch.int16, device="cuda")
     kview = kbuf[frame_elems:(slots + 1) * frame_elems].view(torch.bfloat16).view(slots, F, H, D)
@@ -44,7 +44,7 @@ def run_ring_rope(slots, grid_h, grid_w, H, inserts, seed, stride_mult=1, t_star
         vw[:, :H * D] = vb
         kd = to_dev(kw).view(n * F, stride_mult * H, D)[:, :H, :]
         vd = to_dev(vw).view(n * F, stride_mult * H, D)[:, :H, :]
-        kr = f64_to_bf16_bits(rope3d_ref(bf16_bits_to_f64(kb.reshape(n * F, H, D)), t, grid_h, grid_w))
+        kr = f64_to_bf16_bits(rope3d_ref(bf16_bits_to_f64(kb.reshape(n * F, H, D)), t, grid_h, grid_w, pairs))
         kr = kr.reshape(n * F, H * D)
         frames = [(kr[i * F:(i + 1) * F], vb[i * F:(i + 1) * F], t + i) for i in range(n)]
         ev = rkv.kvcache_ring_update_rope(ring, kd, vd, t, rope, n)
@@ -106,6 +106,11 @@ def test_ring_rope_wide_grid():
 def test_ring_rope_one_row_grid():
     # a 1x4000 grid: a table of every position would need 84,000 entries
     run_ring_rope(3, 1, 4000, 1, [2, 2], seed=79)
+
+
+def test_ring_rope_chunk_on_three_axes():
+    # pairs 21/2/41: rotary pairs 20-23 (one 16-byte chunk) lie on t, h, h, w
+    run_ring_rope(5, 3, 4, 2, [2, 3, 1, 2], seed=80, pairs=(21, 2, 41))
 
 
 def test_ring_rope_rejects_grid_mismatch():

@@ -70,5 +70,13 @@ def test_other_axis_split():
     check_rope(300, 2, 5, 7, 1, 17, pairs=(32, 16, 16))
 
 
+def test_chunk_on_three_axes():
+    # splits where one 16-byte chunk (rotary pairs 4c..4c+3) holds pairs of
+    # t, h and w: chunk 5 = t | h h | w; chunk 0 = t | h | w w; chunk 1 = t | h | w w
+    check_rope(500, 2, 5, 7, 1, 19, pairs=(21, 2, 41))
+    check_rope(500, 2, 5, 7, 1, 20, pairs=(1, 1, 62))
+    check_rope(500, 2, 5, 7, 1, 21, pairs=(5, 1, 58))
+
+
 def test_large_time_index():
     check_rope(200, 2, 4, 6, 1000, 18)
