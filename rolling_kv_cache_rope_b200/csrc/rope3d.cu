@@ -46,7 +46,7 @@ struct RopeArgs {
   int32_t t0;
   int32_t grid_h, grid_w;
   int32_t pt, ph, pw;      // rotary pairs per axis
-  double log2_theta[3];    // per axis t, h, w
+  double omega[64];        // frequency of rotary pair j: theta_a^(-i/count_a), i its index on axis a
   FastDiv div_F, div_W, div_cpr, div_cph;
   // adjacent layout: axis a owns rotary pairs [ax_first[a], + ax_count[a]),
   // i.e. 16-byte chunks [ax_chunk0[a], + ax_nch[a]).  Chunk g's four pairs lie
@@ -65,6 +65,10 @@ constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
 constexpr int kRopeMaxEntries = 4096;  // 64 KB of per-pair entries per CTA (rotate-half)
 constexpr int kAdjMaxEntries = 1024;   // 64 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
+
+__device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z) {
+  return a == 0 ? x : (a == 1 ? y : z);
+}
 
 struct TabEntry {
   float c_hi, s_hi, c_lo, s_lo;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(rope_threads<kRing>()) rope3d_half_kernel(cons
       if (pos >= a.grid_w) pos -= a.grid_w;
     }
     const int axis = e < base_h ? 0 : (e < base_w ? 1 : 2);
-    const double ang = double(pos) * exp2(-(double(i) / double(n)) * a.log2_theta[axis]);
+    const double ang = double(pos) * a.omega[pick3i(axis, 0, a.pt, a.pt + a.ph) + i];
     double s, c;
     sincos(ang, &s, &c);
     TabEntry t;
@@ -303,10 +307,6 @@ __device__ __noinline__ uint4 rotate4_exact(uint4 v, float4 C, float4 S, float4 
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z) {
-  return a == 0 ? x : (a == 1 ? y : z);
-}
-
 // Table entry of 16-byte chunk `chunk` (rotary pairs 4*chunk .. +3) at
 // positions (p_t, p_h, p_w): cos and sin of each pair's angle rounded to
 // fp32 (hi) and the fp32 rounding of the rest (lo).  Pairs on an axis outside
@@ -318,10 +318,8 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
   for (int q = 0; q < 4; ++q) {
     const int32_t pr = 4 * chunk + q;
     const int ax = pr < a.ax_first[1] ? 0 : (pr < a.ax_first[2] ? 1 : 2);
-    const int32_t i = pr - a.ax_first[ax];
     double sd = 0.0, cd = 1.0;
-    if ((axes >> ax) & 1)
-      sincos(double(pick3i(ax, p_t, p_h, p_w)) * exp2(-(double(i) / double(a.ax_count[ax])) * a.log2_theta[ax]), &sd, &cd);
+    if ((axes >> ax) & 1) sincos(double(pick3i(ax, p_t, p_h, p_w)) * a.omega[pr], &sd, &cd);
     c4[q] = __double2float_rn(cd);
     s4[q] = __double2float_rn(sd);
     cl4[q] = __double2float_rn(cd - double(c4[q]));
@@ -339,8 +337,11 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
 // tab_base[a] + k * npos[a] + i holds the 4 pairs of chunk ax_chunk0[a] + k
 // (pairs of that chunk outside axis a hold cos 1, sin 0); a chunk whose pairs
 // lie on several axes instead reads entry (region m, row r - r0) after those,
-// built for each of the CTA's rows.  So every chunk reads one entry, and the
-// threads of a warp take the same path whatever chunk positions they hold.
+// built for each of the CTA's rows as the product of the single-axis entries
+// (exact: each pair has one factor other than cos 1 / sin 0).  So every chunk
+// reads one entry, and the threads of a warp take the same path whatever
+// chunk positions they hold.  The first rows' loads are issued before the
+// table is built, so their latency overlaps the fp64 sincos.
 template <bool kRing>
 __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   extern __shared__ float4 tab4[];
@@ -374,46 +375,72 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   float4* tS = tab4 + E;
   float4* tCl = tab4 + 2 * E;
   float4* tSl = tab4 + 3 * E;
-  for (int32_t e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t pos[3], chunk;
-    int axes;
-    if (e < tbm) {
-      const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
-      const int32_t np = pick3i(ax, npos0, npos1, npos2);
-      const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
-      const int32_t k = rel / np, pi = rel - k * np;
-      int32_t ps = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
-      if (ax == 2 && ps >= a.grid_w) ps -= a.grid_w;
-      pos[0] = pos[1] = pos[2] = ps;
-      chunk = a.ax_chunk0[ax] + k;
-      axes = 1 << ax;
-    } else {
-      // multi-axis chunk: the m-th such chunk position at row r
-      const int32_t m = (e - tbm) / nrows;
-      const uint32_t r = r0 + uint32_t(e - tbm - m * nrows);
-      const uint32_t f = fdiv(r, a.div_F);
-      const uint32_t in_f = r - f * a.F;
-      const uint32_t hh = fdiv(in_f, a.div_W);
-      pos[0] = a.t0 + int32_t(f);
-      pos[1] = int32_t(hh);
-      pos[2] = int32_t(in_f - hh * uint32_t(a.grid_w));
-      chunk = 0;
-      for (int g = 0, seen = 0; g < 16; ++g)
-        if (a.ch_axis[g] < 0 && seen++ == m) chunk = g;
-      axes = 7;
-    }
-    adj_entry(a, chunk, axes, pos[0], pos[1], pos[2], tC[e], tS[e], tCl[e], tSl[e]);
-  }
-  __syncthreads();
-
   // thread -> (chunk position c of a row, row phase rsub): `lanes` threads per
   // row, rpp rows side by side; each thread walks rows r0 + rsub, + rpp, ...
   const uint32_t T = blockDim.x;
   const uint32_t lanes = a.cpr < T ? a.cpr : T;
   const uint32_t rpp = T / lanes;
   const uint32_t rsub = threadIdx.x / lanes;
-  if (rsub >= rpp) return;
-  for (uint32_t c = threadIdx.x - rsub * lanes; c < a.cpr; c += lanes) {
+  const uint32_t c0 = threadIdx.x - rsub * lanes;
+  const bool active = rsub < rpp;
+  // the first rows' loads go out before the table is built
+  uint4 v[kRopeUnroll];
+  if (active) {
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const uint32_t r = r0 + rsub + u * rpp;
+      if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c0) * 16u);
+    }
+  }
+  // single-axis entries (fp64 sincos), then the per-row entries of chunks on
+  // several axes as products of those (each pair has one factor other than
+  // cos 1 / sin 0, so the product and the sums are exact)
+  for (int32_t e = threadIdx.x; e < tbm; e += blockDim.x) {
+    const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
+    const int32_t np = pick3i(ax, npos0, npos1, npos2);
+    const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
+    const int32_t k = rel / np, pi = rel - k * np;
+    int32_t ps = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
+    if (ax == 2 && ps >= a.grid_w) ps -= a.grid_w;
+    adj_entry(a, a.ax_chunk0[ax] + k, 1 << ax, ps, ps, ps, tC[e], tS[e], tCl[e], tSl[e]);
+  }
+  if (a.n_multi > 0) {
+    __syncthreads();
+    for (int32_t e = tbm + int32_t(threadIdx.x); e < E; e += blockDim.x) {
+      const int32_t m = (e - tbm) / nrows;
+      const uint32_t r = r0 + uint32_t(e - tbm - m * nrows);
+      const uint32_t f = fdiv(r, a.div_F);
+      const uint32_t in_f = r - f * a.F;
+      const uint32_t hh = fdiv(in_f, a.div_W);
+      int32_t wi = int32_t(in_f - hh * uint32_t(a.grid_w)) - w_lo;
+      if (wi < 0) wi += a.grid_w;
+      const int32_t idx[3] = {int32_t(f - f_lo), int32_t(hh) - h_lo, wi};
+      int32_t g = 0;
+      for (int gg = 0, seen = 0; gg < 16; ++gg)
+        if (a.ch_axis[gg] < 0 && seen++ == m) g = gg;
+      float4 C = make_float4(1.f, 1.f, 1.f, 1.f), S = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 Cl = S, Sl = S;
+#pragma unroll
+      for (int ax = 0; ax < 3; ++ax) {
+        const int32_t k = g - a.ax_chunk0[ax];
+        if (k < 0 || k >= a.ax_nch[ax]) continue;
+        const int32_t ea = pick3i(ax, tb0, tb1, tb2) + k * pick3i(ax, npos0, npos1, npos2) + idx[ax];
+        const float4 c = tC[ea], s4 = tS[ea], cl = tCl[ea], sl = tSl[ea];
+        C = make_float4(C.x * c.x, C.y * c.y, C.z * c.z, C.w * c.w);
+        S = make_float4(S.x + s4.x, S.y + s4.y, S.z + s4.z, S.w + s4.w);
+        Cl = make_float4(Cl.x + cl.x, Cl.y + cl.y, Cl.z + cl.z, Cl.w + cl.w);
+        Sl = make_float4(Sl.x + sl.x, Sl.y + sl.y, Sl.z + sl.z, Sl.w + sl.w);
+      }
+      tC[e] = C;
+      tS[e] = S;
+      tCl[e] = Cl;
+      tSl[e] = Sl;
+    }
+  }
+  __syncthreads();
+
+  if (!active) return;
+  for (uint32_t c = c0; c < a.cpr; c += lanes) {
     // entry of row r: eb + ti*mt + hi*mh + wi*mw + r*mr, one term non-zero
     const int32_t g = int32_t(c & 15u);
     const int ax = a.ch_axis[g];
@@ -428,11 +455,12 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
       mr = 1;
     }
     for (uint32_t rb = r0 + rsub; rb < r1; rb += rpp * kRopeUnroll) {
-      uint4 v[kRopeUnroll];
+      if (c != c0 || rb != r0 + rsub) {
 #pragma unroll
-      for (int u = 0; u < kRopeUnroll; ++u) {
-        const uint32_t r = rb + u * rpp;
-        if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c) * 16u);
+        for (int u = 0; u < kRopeUnroll; ++u) {
+          const uint32_t r = rb + u * rpp;
+          if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c) * 16u);
+        }
       }
 #pragma unroll
       for (int u = 0; u < kRopeUnroll; ++u) {
@@ -492,9 +520,16 @@ static void fill_rope_args(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const 
   a.pt = rope->pairs_t;
   a.ph = rope->pairs_h;
   a.pw = rope->pairs_w;
-  a.log2_theta[0] = log2(double(rope->theta));
-  a.log2_theta[1] = log2(double(rope->theta_h != 0.0f ? rope->theta_h : rope->theta));
-  a.log2_theta[2] = log2(double(rope->theta_w != 0.0f ? rope->theta_w : rope->theta));
+  {
+    // computed once here (fp64) instead of in every table entry on the device
+    const double log2_theta[3] = {log2(double(rope->theta)),
+                                  log2(double(rope->theta_h != 0.0f ? rope->theta_h : rope->theta)),
+                                  log2(double(rope->theta_w != 0.0f ? rope->theta_w : rope->theta))};
+    const int32_t cnt[3] = {rope->pairs_t, rope->pairs_h, rope->pairs_w};
+    for (int ax = 0, j = 0; ax < 3; ++ax)
+      for (int32_t i = 0; i < cnt[ax] && j < 64; ++i, ++j)
+        a.omega[j] = exp2(-(double(i) / double(cnt[ax])) * log2_theta[ax]);
+  }
   a.cph = uint32_t(H) * 8u;
   a.div_cph = make_fastdiv(a.cph);
   a.div_F = make_fastdiv(a.F);
