@@ -406,7 +406,10 @@ rkv_status kvcache_ring_update(rkv_ring* ring, const void* k_new, const void* v_
  * The ring's K slots receive exactly what rope3d_apply(k_new) would write
  * (same arithmetic, same rounding, within 1 bf16 ulp of the exact rotation);
  * V slots receive v_new unchanged.  Slot, head, count and eviction follow
- * kvcache_ring_update.
+ * kvcache_ring_update.  With the adjacent layout V moves on the TMA
+ * bulk-copy engine as in kvcache_ring_update (same bounded waits: a wait that
+ * gives up sets the flag rkv_ring_status reports, and the insert's slots may
+ * be partly written) while the other threads of each CTA rotate K.
  * Errors: those of kvcache_ring_update and rope3d_apply, plus
  * RKV_ERR_INVALID_ARG when the frame grid does not match tokens_per_frame.
  */

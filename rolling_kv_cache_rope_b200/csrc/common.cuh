@@ -42,6 +42,7 @@ struct RingPlan {
   int32_t n_pin, pin_base, head, end, len;
 };
 RingPlan ring_plan(const rkv_ring* ring);  // ring_update.cu; for a checked ring
+rkv_status ring_timeout_flag(int32_t** out);  // ring_update.cu: this device's ring timeout flag
 
 __host__ __device__ __forceinline__ int32_t ring_dst_slot(const RingPlan& p, uint32_t frame) {
   const int32_t f = int32_t(frame);

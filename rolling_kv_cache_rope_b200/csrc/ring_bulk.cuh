@@ -92,12 +92,43 @@ __device__ __forceinline__ void bulk_store_piece(const RingPiece& pc, uint32_t s
   ptx::bulk_commit();
 }
 
-// This CTA's pieces: local piece i is piece blockIdx.x + i * G of the insert.
-__device__ __forceinline__ uint32_t cta_pieces(uint32_t total, uint32_t G) {
-  return total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0;
-}
-__device__ __forceinline__ RingPiece cta_piece(const RingBulkArgs& a, uint32_t i) {
-  return ring_piece(a, blockIdx.x + i * gridDim.x);
+// One thread moves pieces first, first + G, first + 2G, ... (below end) of
+// the insert through the `a.stages` stages at shared address smem0, piece i
+// of the list in stage i % stages, i.e. phase (i / stages) & 1 of mbarrier
+// full[i % stages] (initialised here).  When a wait gives up it sets
+// a.timeout_flag, lets the loads still in flight land (bounded) and stops.
+__device__ __forceinline__ void bulk_copy_pieces(const RingBulkArgs& a, uint32_t first, uint32_t end, uint32_t G,
+                                                 uint32_t smem0, uint64_t* full) {
+  const uint32_t n = end > first ? (end - first + G - 1) / G : 0u;
+  for (uint32_t s = 0; s < a.stages; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+  ptx::fence_mbar_init();
+  auto piece = [&](uint32_t i) { return ring_piece(a, first + i * G); };
+  auto stage = [&](uint32_t i) { return smem0 + (i % a.stages) * a.stage_bytes; };
+  auto bar = [&](uint32_t i) { return ptx::smem_u32(&full[i % a.stages]); };
+  uint32_t issued = 0;
+  for (; issued < n && issued < a.stages; ++issued)
+    bulk_load_piece(a, piece(issued), stage(issued), bar(issued),
+                    (a.stall && blockIdx.x == 0 && issued == 0) ? 16u : 0u);
+  uint32_t i = 0;
+  for (; i < n; ++i) {
+    if (!bulk_wait(bar(i), (i / a.stages) & 1u, a.wait_ns)) {
+      atomicExch(a.timeout_flag, 1);
+      break;
+    }
+    bulk_store_piece(piece(i), stage(i));
+    // refill the previous piece's stage once its store has read shared memory
+    // (issued == i - 1 + stages here)
+    if (i >= 1 && issued < n) {
+      ptx::bulk_wait_read<1>();
+      bulk_load_piece(a, piece(issued), stage(issued), bar(issued));
+      ++issued;
+    }
+  }
+  // after a wait gave up on piece i: let the loads still in flight, piece i's
+  // included, land (bounded) before the CTA's shared memory is released
+  // (issued <= i + stages, so these pieces use distinct stages)
+  for (uint32_t j = i; j < issued; ++j) bulk_wait(bar(j), (j / a.stages) & 1u, a.wait_ns);
+  ptx::bulk_wait_all();
 }
 
 // Piece geometry of an insert into a checked ring (timeout_flag left null,

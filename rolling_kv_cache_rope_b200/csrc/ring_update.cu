@@ -26,42 +26,12 @@ namespace rkv {
 
 constexpr int kBulkThreads = 32;
 
-// Piece i of this CTA is staged in slot i % stages, i.e. phase
-// (i / stages) & 1 of that slot's mbarrier.
+// CTA b moves pieces b, b + G, b + 2G, ... of the insert (K pieces, then V).
 __global__ void __launch_bounds__(kBulkThreads, 1) ring_bulk_kernel(const RingBulkArgs a) {
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t full[kBulkStages];
   if (threadIdx.x != 0) return;
-  const uint32_t n = cta_pieces(a.total, gridDim.x);
-  const uint32_t smem0 = ptx::smem_u32(stage_mem);
-  for (uint32_t s = 0; s < a.stages; ++s) ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
-  ptx::fence_mbar_init();
-  auto stage = [&](uint32_t i) { return smem0 + (i % a.stages) * a.stage_bytes; };
-  auto bar = [&](uint32_t i) { return ptx::smem_u32(&full[i % a.stages]); };
-  uint32_t issued = 0;
-  for (; issued < n && issued < a.stages; ++issued)
-    bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued),
-                    (a.stall && blockIdx.x == 0 && issued == 0) ? 16u : 0u);
-  uint32_t i = 0;
-  for (; i < n; ++i) {
-    if (!bulk_wait(bar(i), (i / a.stages) & 1u, a.wait_ns)) {
-      atomicExch(a.timeout_flag, 1);
-      break;
-    }
-    bulk_store_piece(cta_piece(a, i), stage(i));
-    // refill the previous piece's stage once its store has read shared memory
-    // (issued == i - 1 + stages here)
-    if (i >= 1 && issued < n) {
-      ptx::bulk_wait_read<1>();
-      bulk_load_piece(a, cta_piece(a, issued), stage(issued), bar(issued));
-      ++issued;
-    }
-  }
-  // after a wait gave up on piece i: let the loads still in flight, piece i's
-  // included, land (bounded) before the CTA's shared memory is released
-  // (issued <= i + stages, so these pieces use distinct stages)
-  for (uint32_t j = i; j < issued; ++j) bulk_wait(bar(j), (j / a.stages) & 1u, a.wait_ns);
-  ptx::bulk_wait_all();
+  bulk_copy_pieces(a, blockIdx.x, a.total, gridDim.x, ptx::smem_u32(stage_mem), full);
 }
 
 static int sm_count() {
@@ -144,7 +114,7 @@ static __device__ int32_t g_ring_timeout;
 static std::mutex g_ring_mu;
 static int32_t* g_ring_timeout_ptr[kMaxDevices];
 
-static rkv_status ring_timeout_flag(int32_t** out) {
+rkv_status ring_timeout_flag(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");

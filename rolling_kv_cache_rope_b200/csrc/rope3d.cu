@@ -22,11 +22,18 @@
 // bytes of table, and the exact path is out of line.  A chunk whose pairs lie
 // on two or three axes reads per-row entries, so every chunk takes the same
 // path.  Rotate-half pairs (rope3d_half_kernel) keep the per-pair table.
+//
+// Rotated ring insert, adjacent pairs (ring_rope_kernel): one CTA per SM; one
+// thread moves V on the TMA bulk-copy engine exactly as kvcache_ring_update
+// does, the other warps build the table and rotate K into the ring, so the
+// table build and the rotation run under V's copy.
 #include <math.h>
 
 #include <algorithm>
 
 #include "common.cuh"
+#include "ring_bulk.cuh"
+#include "sm100_ptx.cuh"
 
 namespace rkv {
 
@@ -65,6 +72,8 @@ constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
 constexpr int kRopeMaxEntries = 4096;  // 64 KB of per-pair entries per CTA (rotate-half)
 constexpr int kAdjMaxEntries = 1024;   // 64 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
+constexpr int kRingRopeThreads = 640;   // rotated ring insert, at most: warp 0 copies V, the rest rotate K
+constexpr int kRingRopeSmem = 227 * 1024 - 256;   // its dynamic shared memory at most (V stages + table)
 
 __device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z) {
   return a == 0 ? x : (a == 1 ? y : z);
@@ -342,16 +351,18 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
 // reads one entry, and the threads of a warp take the same path whatever
 // chunk positions they hold.  The first rows' loads are issued before the
 // table is built, so their latency overlaps the fp64 sincos.
+// Rows [r0, r1) by threads tid = 0 .. T-1 of the CTA (table in tab4); bar = 0
+// synchronises with __syncthreads, else with named barrier `bar` over the T
+// threads.
 template <bool kRing>
-__global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
-  extern __shared__ float4 tab4[];
-  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
-  if (r0 >= a.L) return;
-  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
-  if (kRing && blockIdx.y == 1) {
-    copy_rows_to_ring(a, r0, r1);
-    return;
-  }
+__device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint32_t r1, uint32_t tid, uint32_t T,
+                                           float4* tab4, uint32_t bar) {
+  auto sync = [&]() {
+    if (bar == 0)
+      __syncthreads();
+    else
+      ptx::named_sync_and(bar, T, true);
+  };
   // positions this CTA's rows reach: frames f_lo..f_hi; grid rows
   // h_lo..h_lo+nh-1; columns w_lo, w_lo+1, ... (mod grid_w), nw of them
   const uint32_t f_lo = fdiv(r0, a.div_F), f_hi = fdiv(r1 - 1, a.div_F);
@@ -377,11 +388,10 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   float4* tSl = tab4 + 3 * E;
   // thread -> (chunk position c of a row, row phase rsub): `lanes` threads per
   // row, rpp rows side by side; each thread walks rows r0 + rsub, + rpp, ...
-  const uint32_t T = blockDim.x;
   const uint32_t lanes = a.cpr < T ? a.cpr : T;
   const uint32_t rpp = T / lanes;
-  const uint32_t rsub = threadIdx.x / lanes;
-  const uint32_t c0 = threadIdx.x - rsub * lanes;
+  const uint32_t rsub = tid / lanes;
+  const uint32_t c0 = tid - rsub * lanes;
   const bool active = rsub < rpp;
   // the first rows' loads go out before the table is built
   uint4 v[kRopeUnroll];
@@ -395,7 +405,7 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   // single-axis entries (fp64 sincos), then the per-row entries of chunks on
   // several axes as products of those (each pair has one factor other than
   // cos 1 / sin 0, so the product and the sums are exact)
-  for (int32_t e = threadIdx.x; e < tbm; e += blockDim.x) {
+  for (int32_t e = int32_t(tid); e < tbm; e += int32_t(T)) {
     const int ax = e < tb1 ? 0 : (e < tb2 ? 1 : 2);
     const int32_t np = pick3i(ax, npos0, npos1, npos2);
     const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
@@ -405,8 +415,8 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
     adj_entry(a, a.ax_chunk0[ax] + k, 1 << ax, ps, ps, ps, tC[e], tS[e], tCl[e], tSl[e]);
   }
   if (a.n_multi > 0) {
-    __syncthreads();
-    for (int32_t e = tbm + int32_t(threadIdx.x); e < E; e += blockDim.x) {
+    sync();
+    for (int32_t e = tbm + int32_t(tid); e < E; e += int32_t(T)) {
       const int32_t m = (e - tbm) / nrows;
       const uint32_t r = r0 + uint32_t(e - tbm - m * nrows);
       const uint32_t f = fdiv(r, a.div_F);
@@ -437,7 +447,7 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
       tSl[e] = Sl;
     }
   }
-  __syncthreads();
+  sync();
 
   if (!active) return;
   for (uint32_t c = c0; c < a.cpr; c += lanes) {
@@ -482,6 +492,40 @@ __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
       }
     }
   }
+}
+
+template <bool kRing>
+__global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
+  extern __shared__ float4 tab4[];
+  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
+  if (r0 >= a.L) return;
+  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
+  if (kRing && blockIdx.y == 1) {
+    copy_rows_to_ring(a, r0, r1);
+    return;
+  }
+  adj_rotate<kRing>(a, r0, r1, threadIdx.x, blockDim.x, tab4, 0);
+}
+
+// Rotated ring insert (adjacent layout), one CTA per SM: one thread of warp 0
+// moves the CTA's share of the V pieces on the TMA bulk-copy engine (global ->
+// shared memory -> ring slot, the kvcache_ring_update path), while warps
+// 1..31 build the cos/sin table and rotate the CTA's block of K rows through
+// registers into the ring: the table build and the rotation run under V's
+// copy.  Shared memory: V stages, then the table.  Fewer threads than the
+// standalone kernel keep its registers (the V copy needs none of them).
+__global__ void __launch_bounds__(kRingRopeThreads, 1) ring_rope_kernel(const RopeArgs a, const RingBulkArgs vb) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kBulkStages];
+  if (threadIdx.x < 32) {
+    if (threadIdx.x == 0) bulk_copy_pieces(vb, vb.half + blockIdx.x, vb.total, gridDim.x, ptx::smem_u32(smem), full);
+    return;
+  }
+  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
+  if (r0 >= a.L) return;
+  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
+  adj_rotate<true>(a, r0, r1, threadIdx.x - 32, blockDim.x - 32,
+                   reinterpret_cast<float4*>(smem + vb.stages * vb.stage_bytes), 1);
 }
 
 static int sm_count() {
@@ -586,7 +630,7 @@ static rkv_status launch_rope_half(RopeArgs& a, int64_t L, cudaStream_t stream) 
 // standalone op, one CTA per SM) or in 256 threads (the ring insert, four
 // CTAs per SM beside the V copy); rows per CTA under the table budget.
 template <bool kRing>
-static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
+static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, const RingBulkArgs* vb, cudaStream_t stream) {
   const int64_t lanes = std::min<int64_t>(a.cpr, 1024);
   const int64_t cap = kRing ? 256 : 1024;
   const int64_t threads = lanes * std::max<int64_t>(1, cap / lanes);
@@ -600,6 +644,32 @@ static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
            int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows) + int64_t(a.n_multi) * rows;
   };
   if (entries(1) > kAdjMaxEntries) return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
+  if (kRing && vb) {
+    // one CTA per SM; V stages beside the table
+    int64_t r = (L + sm_count() - 1) / sm_count();
+    if (r < 1) r = 1;
+    while (r > 1 && entries(r) > kAdjMaxEntries) r = (r + 1) / 2;
+    const int64_t table = entries(r) * 4 * int64_t(sizeof(float4));
+    const int64_t stages = std::min<int64_t>(kBulkStages, (kRingRopeSmem - table) / vb->stage_bytes);
+    if (stages >= 2) {
+      RingBulkArgs v = *vb;
+      v.stages = uint32_t(stages);
+      a.rows_per_cta = uint32_t(r);
+      const int64_t grid = (L + r - 1) / r;
+      const int smem = int(stages * v.stage_bytes + table);
+      cudaError_t e = cudaFuncSetAttribute(ring_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingRopeSmem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(ring_rope_kernel)");
+      // rotating threads: whole rows of chunks, rounded up to whole warps (the
+      // named barrier counts warps; the extra threads only join it)
+      const int64_t lanes = std::min<int64_t>(a.cpr, kRingRopeThreads - 32);
+      const int64_t rot = lanes * std::max<int64_t>(1, (kRingRopeThreads - 32) / lanes);
+      const int64_t threads = 32 + (rot + 31) / 32 * 32;
+      ring_rope_kernel<<<uint32_t(grid), uint32_t(threads), smem, stream>>>(a, v);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "ring_rope_kernel launch");
+      return RKV_OK;
+    }
+  }
   while (rpc > 1 && entries(rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
   a.rows_per_cta = uint32_t(rpc);
   const int64_t grid = (L + rpc - 1) / rpc;
@@ -615,9 +685,10 @@ static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
 
 template <bool kRing>
 static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
-                              cudaStream_t stream) {
+                              const RingBulkArgs* vb, cudaStream_t stream) {
   fill_rope_args(a, L, H, t0, rope);
-  return rope->layout == RKV_ROPE_HALF ? launch_rope_half<kRing>(a, L, stream) : launch_rope_adj<kRing>(a, L, stream);
+  return rope->layout == RKV_ROPE_HALF ? launch_rope_half<kRing>(a, L, stream)
+                                       : launch_rope_adj<kRing>(a, L, vb, stream);
 }
 
 }  // namespace rkv
@@ -652,7 +723,7 @@ extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H,
   a.y = static_cast<uint8_t*>(y);
   a.x_stride_bytes = x_row_stride * 2;
   a.y_stride_bytes = y_row_stride * 2;
-  return launch_rope<false>(a, L, H, t0, rope, static_cast<cudaStream_t>(stream));
+  return launch_rope<false>(a, L, H, t0, rope, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
@@ -680,7 +751,13 @@ extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new
     a.y_stride_bytes = int64_t(ring->H) * ring->D * 2;
     a.slot_bytes = uint64_t(ring->tokens_per_frame) * ring->H * ring->D * 2;
     a.ring = ring_plan(ring);
-    st = launch_rope<true>(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope,
+    // V goes through the bulk-copy pieces of a plain insert (the V half)
+    RingBulkArgs vb;
+    st = ring_bulk_geometry(ring, k_new, v_new, new_row_stride, n_frames, vb);
+    if (st != RKV_OK) return st;
+    st = ring_timeout_flag(&vb.timeout_flag);
+    if (st != RKV_OK) return st;
+    st = launch_rope<true>(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope, &vb,
                            static_cast<cudaStream_t>(stream));
     if (st != RKV_OK) return st;
   }
