@@ -340,7 +340,7 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
   Sl = make_float4(sl4[0], sl4[1], sl4[2], sl4[3]);
 }
 
-// Adjacent layout (pairs 2j, 2j+1).  kRing as rope3d_half_kernel.  Table
+// Adjacent layout (pairs 2j, 2j+1).  kRing: K rows go to their ring slots.  Table
 // (shared memory, four float4 arrays of E entries: cos hi, sin hi, cos lo,
 // sin lo).  Entry (axis a, chunk k of the axis, position index i) at
 // tab_base[a] + k * npos[a] + i holds the 4 pairs of chunk ax_chunk0[a] + k
@@ -351,6 +351,7 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
 // reads one entry, and the threads of a warp take the same path whatever
 // chunk positions they hold.  The first rows' loads are issued before the
 // table is built, so their latency overlaps the fp64 sincos.
+//
 // Rows [r0, r1) by threads tid = 0 .. T-1 of the CTA (table in tab4); bar = 0
 // synchronises with __syncthreads, else with named barrier `bar` over the T
 // threads.
@@ -494,17 +495,13 @@ __device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint3
   }
 }
 
-template <bool kRing>
+// Standalone op (adjacent layout): one CTA per SM over a block of rows.
 __global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
   extern __shared__ float4 tab4[];
   const uint32_t r0 = blockIdx.x * a.rows_per_cta;
   if (r0 >= a.L) return;
   const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
-  if (kRing && blockIdx.y == 1) {
-    copy_rows_to_ring(a, r0, r1);
-    return;
-  }
-  adj_rotate<kRing>(a, r0, r1, threadIdx.x, blockDim.x, tab4, 0);
+  adj_rotate<false>(a, r0, r1, threadIdx.x, blockDim.x, tab4, 0);
 }
 
 // Rotated ring insert (adjacent layout), one CTA per SM: one thread of warp 0
@@ -625,61 +622,63 @@ static rkv_status launch_rope_half(RopeArgs& a, int64_t L, cudaStream_t stream) 
   return RKV_OK;
 }
 
-// Adjacent layout: a block is `lanes` threads per row (one per 16-byte chunk,
-// at most 1024) times the rows side by side that fit in 1024 threads (the
-// standalone op, one CTA per SM) or in 256 threads (the ring insert, four
-// CTAs per SM beside the V copy); rows per CTA under the table budget.
-template <bool kRing>
-static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, const RingBulkArgs* vb, cudaStream_t stream) {
+// upper bound of the chunk entries a CTA of `rows` rows builds (see adj_rotate)
+static int64_t adj_entries(const RopeArgs& a, int64_t rows) {
+  const int64_t nt = rows / a.F + 2;
+  return int64_t(a.ax_nch[0]) * nt + int64_t(a.ax_nch[1]) * a.grid_h +
+         int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows) + int64_t(a.n_multi) * rows;
+}
+
+// Adjacent layout, standalone: `lanes` threads per row (one per 16-byte
+// chunk, at most 1024) times the rows side by side that fit in 1024 threads,
+// one CTA per SM; rows per CTA under the table budget.
+static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
+  if (adj_entries(a, 1) > kAdjMaxEntries)
+    return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
   const int64_t lanes = std::min<int64_t>(a.cpr, 1024);
-  const int64_t cap = kRing ? 256 : 1024;
-  const int64_t threads = lanes * std::max<int64_t>(1, cap / lanes);
-  const int64_t target_ctas = int64_t(sm_count()) * (kRing ? 4 : 1);
-  int64_t rpc = (L + target_ctas - 1) / target_ctas;
+  const int64_t threads = lanes * std::max<int64_t>(1, 1024 / lanes);
+  int64_t rpc = (L + sm_count() - 1) / sm_count();
   if (rpc < 1) rpc = 1;
-  // upper bound of the chunk entries a CTA of `rows` rows builds (see the kernel)
-  auto entries = [&](int64_t rows) {
-    const int64_t nt = rows / a.F + 2;
-    return int64_t(a.ax_nch[0]) * nt + int64_t(a.ax_nch[1]) * a.grid_h +
-           int64_t(a.ax_nch[2]) * std::min<int64_t>(a.grid_w, rows) + int64_t(a.n_multi) * rows;
-  };
-  if (entries(1) > kAdjMaxEntries) return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
-  if (kRing && vb) {
-    // one CTA per SM; V stages beside the table
-    int64_t r = (L + sm_count() - 1) / sm_count();
-    if (r < 1) r = 1;
-    while (r > 1 && entries(r) > kAdjMaxEntries) r = (r + 1) / 2;
-    const int64_t table = entries(r) * 4 * int64_t(sizeof(float4));
-    const int64_t stages = std::min<int64_t>(kBulkStages, (kRingRopeSmem - table) / vb->stage_bytes);
-    if (stages >= 2) {
-      RingBulkArgs v = *vb;
-      v.stages = uint32_t(stages);
-      a.rows_per_cta = uint32_t(r);
-      const int64_t grid = (L + r - 1) / r;
-      const int smem = int(stages * v.stage_bytes + table);
-      cudaError_t e = cudaFuncSetAttribute(ring_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingRopeSmem);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(ring_rope_kernel)");
-      // rotating threads: whole rows of chunks, rounded up to whole warps (the
-      // named barrier counts warps; the extra threads only join it)
-      const int64_t lanes = std::min<int64_t>(a.cpr, kRingRopeThreads - 32);
-      const int64_t rot = lanes * std::max<int64_t>(1, (kRingRopeThreads - 32) / lanes);
-      const int64_t threads = 32 + (rot + 31) / 32 * 32;
-      ring_rope_kernel<<<uint32_t(grid), uint32_t(threads), smem, stream>>>(a, v);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return cuda_fail(e, "ring_rope_kernel launch");
-      return RKV_OK;
-    }
-  }
-  while (rpc > 1 && entries(rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
+  while (rpc > 1 && adj_entries(a, rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
   a.rows_per_cta = uint32_t(rpc);
   const int64_t grid = (L + rpc - 1) / rpc;
-  const size_t smem = size_t(entries(rpc)) * 4 * sizeof(float4);
-  cudaError_t e = cudaFuncSetAttribute(rope3d_adj_kernel<kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = size_t(adj_entries(a, rpc)) * 4 * sizeof(float4);
+  cudaError_t e = cudaFuncSetAttribute(rope3d_adj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAdjMaxEntries * 4 * int(sizeof(float4)));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_adj_kernel)");
-  rope3d_adj_kernel<kRing><<<dim3(uint32_t(grid), kRing ? 2u : 1u), uint32_t(threads), smem, stream>>>(a);
+  rope3d_adj_kernel<<<uint32_t(grid), uint32_t(threads), smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope3d_adj_kernel launch");
+  return RKV_OK;
+}
+
+// Adjacent layout, ring insert: one CTA per SM, its K rows under the table
+// budget, as many V stages as fit beside the table (the table is at most
+// 64 KB, so at least 5 always do).
+static rkv_status launch_ring_rope(RopeArgs& a, int64_t L, const RingBulkArgs& vb, cudaStream_t stream) {
+  if (adj_entries(a, 1) > kAdjMaxEntries)
+    return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
+  int64_t r = (L + sm_count() - 1) / sm_count();
+  if (r < 1) r = 1;
+  while (r > 1 && adj_entries(a, r) > kAdjMaxEntries) r = (r + 1) / 2;
+  const int64_t table = adj_entries(a, r) * 4 * int64_t(sizeof(float4));
+  const int64_t stages = std::min<int64_t>(kBulkStages, (kRingRopeSmem - table) / vb.stage_bytes);
+  if (stages < 2) return fail(RKV_ERR_UNSUPPORTED, "no room for the V stages beside the cos/sin table");
+  RingBulkArgs v = vb;
+  v.stages = uint32_t(stages);
+  a.rows_per_cta = uint32_t(r);
+  const int64_t grid = (L + r - 1) / r;
+  const int smem = int(stages * v.stage_bytes + table);
+  cudaError_t e = cudaFuncSetAttribute(ring_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingRopeSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(ring_rope_kernel)");
+  // rotating threads: whole rows of chunks, rounded up to whole warps (the
+  // named barrier counts warps; the extra threads only join it)
+  const int64_t lanes = std::min<int64_t>(a.cpr, kRingRopeThreads - 32);
+  const int64_t rot = lanes * std::max<int64_t>(1, (kRingRopeThreads - 32) / lanes);
+  const int64_t threads = 32 + (rot + 31) / 32 * 32;
+  ring_rope_kernel<<<uint32_t(grid), uint32_t(threads), smem, stream>>>(a, v);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "ring_rope_kernel launch");
   return RKV_OK;
 }
 
@@ -687,8 +686,8 @@ template <bool kRing>
 static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
                               const RingBulkArgs* vb, cudaStream_t stream) {
   fill_rope_args(a, L, H, t0, rope);
-  return rope->layout == RKV_ROPE_HALF ? launch_rope_half<kRing>(a, L, stream)
-                                       : launch_rope_adj<kRing>(a, L, vb, stream);
+  if (rope->layout == RKV_ROPE_HALF) return launch_rope_half<kRing>(a, L, stream);
+  return kRing ? launch_ring_rope(a, L, *vb, stream) : launch_rope_adj(a, L, stream);
 }
 
 }  // namespace rkv
