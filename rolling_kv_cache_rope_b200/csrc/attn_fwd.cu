@@ -91,6 +91,9 @@ constexpr float kRescaleLog2 = 8.0f; // move the running max only past 2^8 growt
 // four shares add up to the 4 x 128 registers per thread the block launches with
 constexpr int kRegSoftmax = 176, kRegRope = 80, kRegProducer = 80;
 static_assert(2 * kRegSoftmax + kRegRope + kRegProducer == 4 * 128, "register split must match the launch");
+// setmaxnreg.inc may only raise and .dec only lower a warp's count (128 at
+// launch); a .dec above the current count is an illegal instruction
+static_assert(kRegSoftmax >= 128 && kRegRope <= 128 && kRegProducer <= 128, "inc/dec directions of the split");
 
 // shared-memory map (offsets from a 1024-byte aligned base; identical in both CTAs)
 constexpr int kOffQ = 0;
