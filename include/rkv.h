@@ -107,6 +107,40 @@ rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H, int32_t D,
                         int64_t x_row_stride, int64_t y_row_stride, int32_t t0,
                         const rkv_rope3d* rope, void* stream);
 
+/*
+ * rope3d_apply_batch -- rope3d_apply on several tensors (e.g. a layer's Q and
+ * K) that share H, D and rope, in one launch.
+ *
+ * Source: as rope3d_apply; the pages rotate Q and K of the same window
+ * ("Amazon and Reactor tune Trainium for real-time video generation", section
+ * "Three problems for generic compilers").
+ *
+ *   tensors       host array of n descriptors (caller-owned, read during the
+ *                 call): x, y, L, x_row_stride, y_row_stride, t0 exactly as
+ *                 rope3d_apply's arguments of the same names.
+ *   n             0 .. RKV_ROPE_BATCH_MAX (0 = no-op).
+ * Each tensor's y receives what rope3d_apply on that tensor alone would write
+ * (bit-identical).  With the adjacent layout all tensors share one launch
+ * (CTAs shared out by rows); with the rotate-half layout they launch one after
+ * another on `stream`.
+ * Errors: those of rope3d_apply for any tensor, plus RKV_ERR_INVALID_ARG for
+ * n out of range, a NULL array, or an output that overlaps another tensor's
+ * input or output.
+ */
+#define RKV_ROPE_BATCH_MAX 8
+
+typedef struct {
+  const void* x;
+  void* y;
+  int64_t L;
+  int64_t x_row_stride;
+  int64_t y_row_stride;
+  int32_t t0;
+} rkv_rope_tensor;
+
+rkv_status rope3d_apply_batch(const rkv_rope_tensor* tensors, int32_t n, int32_t H, int32_t D,
+                              const rkv_rope3d* rope, void* stream);
+
 /* flags of rkv_attn_seq */
 #define RKV_ROPE_Q 1u /* rotate Q rows by RoPE3D (positions from q_t0) in-kernel */
 #define RKV_ROPE_K 2u /* rotate K rows by RoPE3D (positions from k_t0) in-kernel */

@@ -21,7 +21,9 @@
 // of 4 consecutive pairs at one position, 16 bytes each), so a chunk reads 32
 // bytes of table, and the exact path is out of line.  A chunk whose pairs lie
 // on two or three axes reads per-row entries, so every chunk takes the same
-// path.  Rotate-half pairs (rope3d_half_kernel) keep the per-pair table.
+// path.  One launch covers up to RKV_ROPE_BATCH_MAX tensors
+// (rope3d_apply_batch), CTAs shared out by rows.  Rotate-half pairs
+// (rope3d_half_kernel) keep the per-pair table and launch per tensor.
 //
 // Rotated ring insert, adjacent pairs (ring_rope_kernel): one CTA per SM; one
 // thread moves V on the TMA bulk-copy engine exactly as kvcache_ring_update
@@ -70,10 +72,28 @@ struct RopeArgs {
 template <bool kRing>
 constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
+constexpr int kRopeBatchMax = RKV_ROPE_BATCH_MAX;   // tensors of one rope3d_apply_batch launch
 constexpr int kRopeMaxEntries = 4096;  // 64 KB of per-pair entries per CTA (rotate-half)
 constexpr int kAdjMaxEntries = 1024;   // 64 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
 constexpr int kRingRopeThreads = 640;   // rotated ring insert, at most: warp 0 copies V, the rest rotate K
 constexpr int kRingRopeSmem = 227 * 1024 - 256;   // its dynamic shared memory at most (V stages + table)
+
+// One tensor of a standalone launch: source and destination rows (strides in
+// bytes) and the time index of row 0's frame.
+struct RopeRows {
+  const uint8_t* x;
+  uint8_t* y;
+  int64_t xs, ys;
+  int32_t t0;
+};
+// Tensors of a standalone launch: tensor i holds CTAs [cta0[i], cta0[i + 1]),
+// rpc[i] of its L[i] rows each.
+struct RopeBatch {
+  int32_t n;
+  uint32_t cta0[kRopeBatchMax + 1];
+  uint32_t L[kRopeBatchMax], rpc[kRopeBatchMax];
+  RopeRows t[kRopeBatchMax];
+};
 
 __device__ __forceinline__ int32_t pick3i(int a, int32_t x, int32_t y, int32_t z) {
   return a == 0 ? x : (a == 1 ? y : z);
@@ -356,8 +376,8 @@ __device__ void adj_entry(const RopeArgs& a, int32_t chunk, int axes, int32_t p_
 // synchronises with __syncthreads, else with named barrier `bar` over the T
 // threads.
 template <bool kRing>
-__device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint32_t r1, uint32_t tid, uint32_t T,
-                                           float4* tab4, uint32_t bar) {
+__device__ __forceinline__ void adj_rotate(const RopeArgs& a, const RopeRows rr, uint32_t r0, uint32_t r1, uint32_t tid,
+                                           uint32_t T, float4* tab4, uint32_t bar) {
   auto sync = [&]() {
     if (bar == 0)
       __syncthreads();
@@ -400,7 +420,7 @@ __device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint3
 #pragma unroll
     for (int u = 0; u < kRopeUnroll; ++u) {
       const uint32_t r = r0 + rsub + u * rpp;
-      if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c0) * 16u);
+      if (r < r1) v[u] = *reinterpret_cast<const uint4*>(rr.x + int64_t(r) * rr.xs + uint64_t(c0) * 16u);
     }
   }
   // single-axis entries (fp64 sincos), then the per-row entries of chunks on
@@ -411,7 +431,7 @@ __device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint3
     const int32_t np = pick3i(ax, npos0, npos1, npos2);
     const int32_t rel = e - pick3i(ax, tb0, tb1, tb2);
     const int32_t k = rel / np, pi = rel - k * np;
-    int32_t ps = ax == 0 ? a.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
+    int32_t ps = ax == 0 ? rr.t0 + int32_t(f_lo) + pi : (ax == 1 ? h_lo + pi : w_lo + pi);
     if (ax == 2 && ps >= a.grid_w) ps -= a.grid_w;
     adj_entry(a, a.ax_chunk0[ax] + k, 1 << ax, ps, ps, ps, tC[e], tS[e], tCl[e], tSl[e]);
   }
@@ -470,7 +490,7 @@ __device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint3
 #pragma unroll
         for (int u = 0; u < kRopeUnroll; ++u) {
           const uint32_t r = rb + u * rpp;
-          if (r < r1) v[u] = *reinterpret_cast<const uint4*>(a.x + int64_t(r) * a.x_stride_bytes + uint64_t(c) * 16u);
+          if (r < r1) v[u] = *reinterpret_cast<const uint4*>(rr.x + int64_t(r) * rr.xs + uint64_t(c) * 16u);
         }
       }
 #pragma unroll
@@ -489,19 +509,24 @@ __device__ __forceinline__ void adj_rotate(const RopeArgs& a, uint32_t r0, uint3
         bool bad;
         uint4 out = rotate4(v[u], C, S, bad);
         if (bad) out = rotate4_exact(v[u], C, S, tCl[e], tSl[e]);
-        *reinterpret_cast<uint4*>(dst_chunk<kRing>(a, a.y, r, f, in_f, c)) = out;
+        uint8_t* dst = kRing ? dst_chunk<true>(a, rr.y, r, f, in_f, c) : rr.y + int64_t(r) * rr.ys + uint64_t(c) * 16u;
+        *reinterpret_cast<uint4*>(dst) = out;
       }
     }
   }
 }
 
-// Standalone op (adjacent layout): one CTA per SM over a block of rows.
-__global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a) {
+// Standalone op (adjacent layout): one CTA per SM over a block of rows of
+// one of the launch's tensors (rope3d_apply: one tensor; rope3d_apply_batch:
+// up to kRopeBatchMax, the CTAs shared out by rows).
+__global__ void __launch_bounds__(1024) rope3d_adj_kernel(const RopeArgs a, const RopeBatch b) {
   extern __shared__ float4 tab4[];
-  const uint32_t r0 = blockIdx.x * a.rows_per_cta;
-  if (r0 >= a.L) return;
-  const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
-  adj_rotate<false>(a, r0, r1, threadIdx.x, blockDim.x, tab4, 0);
+  int i = 0;
+  while (i + 1 < b.n && blockIdx.x >= b.cta0[i + 1]) ++i;
+  const uint32_t r0 = (blockIdx.x - b.cta0[i]) * b.rpc[i];
+  if (r0 >= b.L[i]) return;
+  const uint32_t r1 = min(b.L[i], r0 + b.rpc[i]);
+  adj_rotate<false>(a, b.t[i], r0, r1, threadIdx.x, blockDim.x, tab4, 0);
 }
 
 // Rotated ring insert (adjacent layout), one CTA per SM: one thread of warp 0
@@ -521,7 +546,8 @@ __global__ void __launch_bounds__(kRingRopeThreads, 1) ring_rope_kernel(const Ro
   const uint32_t r0 = blockIdx.x * a.rows_per_cta;
   if (r0 >= a.L) return;
   const uint32_t r1 = min(a.L, r0 + a.rows_per_cta);
-  adj_rotate<true>(a, r0, r1, threadIdx.x - 32, blockDim.x - 32,
+  adj_rotate<true>(a, RopeRows{a.x, a.y, a.x_stride_bytes, a.y_stride_bytes, a.t0}, r0, r1, threadIdx.x - 32,
+                   blockDim.x - 32,
                    reinterpret_cast<float4*>(smem + vb.stages * vb.stage_bytes), 1);
 }
 
@@ -631,22 +657,37 @@ static int64_t adj_entries(const RopeArgs& a, int64_t rows) {
 
 // Adjacent layout, standalone: `lanes` threads per row (one per 16-byte
 // chunk, at most 1024) times the rows side by side that fit in 1024 threads,
-// one CTA per SM; rows per CTA under the table budget.
-static rkv_status launch_rope_adj(RopeArgs& a, int64_t L, cudaStream_t stream) {
+// one CTA per SM over all the launch's tensors (each gets CTAs in proportion
+// to its rows, at least one); rows per CTA under the table budget.
+static rkv_status launch_rope_adj(RopeArgs& a, const RopeRows* rows, const int64_t* L, int n, cudaStream_t stream) {
   if (adj_entries(a, 1) > kAdjMaxEntries)
     return fail(RKV_ERR_UNSUPPORTED, "frame grid too large for the on-chip cos/sin table");
   const int64_t lanes = std::min<int64_t>(a.cpr, 1024);
   const int64_t threads = lanes * std::max<int64_t>(1, 1024 / lanes);
-  int64_t rpc = (L + sm_count() - 1) / sm_count();
-  if (rpc < 1) rpc = 1;
-  while (rpc > 1 && adj_entries(a, rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
-  a.rows_per_cta = uint32_t(rpc);
-  const int64_t grid = (L + rpc - 1) / rpc;
-  const size_t smem = size_t(adj_entries(a, rpc)) * 4 * sizeof(float4);
+  int64_t total = 0;
+  for (int i = 0; i < n; ++i) total += L[i];
+  RopeBatch b{};
+  b.n = n;
+  int64_t cta = 0, max_entries = 0;
+  for (int i = 0; i < n; ++i) {
+    int64_t c = std::max<int64_t>(1, (int64_t(sm_count()) * L[i] + total / 2) / total);
+    int64_t rpc = (L[i] + c - 1) / c;
+    while (rpc > 1 && adj_entries(a, rpc) > kAdjMaxEntries) rpc = (rpc + 1) / 2;
+    c = (L[i] + rpc - 1) / rpc;
+    b.cta0[i] = uint32_t(cta);
+    b.L[i] = uint32_t(L[i]);
+    b.rpc[i] = uint32_t(rpc);
+    b.t[i] = rows[i];
+    cta += c;
+    max_entries = std::max<int64_t>(max_entries, adj_entries(a, rpc));
+  }
+  b.cta0[n] = uint32_t(cta);
+  if (cta >= (int64_t(1) << 31)) return fail(RKV_ERR_UNSUPPORTED, "too many rows for one launch");
+  const size_t smem = size_t(max_entries) * 4 * sizeof(float4);
   cudaError_t e = cudaFuncSetAttribute(rope3d_adj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAdjMaxEntries * 4 * int(sizeof(float4)));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rope3d_adj_kernel)");
-  rope3d_adj_kernel<<<uint32_t(grid), uint32_t(threads), smem, stream>>>(a);
+  rope3d_adj_kernel<<<uint32_t(cta), uint32_t(threads), smem, stream>>>(a, b);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope3d_adj_kernel launch");
   return RKV_OK;
@@ -682,12 +723,79 @@ static rkv_status launch_ring_rope(RopeArgs& a, int64_t L, const RingBulkArgs& v
   return RKV_OK;
 }
 
-template <bool kRing>
-static rkv_status launch_rope(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
-                              const RingBulkArgs* vb, cudaStream_t stream) {
+// Rotated ring insert: adjacent layout on ring_rope_kernel, rotate-half on
+// rope3d_half_kernel<true>.
+static rkv_status launch_ring(RopeArgs& a, int64_t L, int32_t H, int32_t t0, const rkv_rope3d* rope,
+                              const RingBulkArgs& vb, cudaStream_t stream) {
   fill_rope_args(a, L, H, t0, rope);
-  if (rope->layout == RKV_ROPE_HALF) return launch_rope_half<kRing>(a, L, stream);
-  return kRing ? launch_ring_rope(a, L, *vb, stream) : launch_rope_adj(a, L, stream);
+  if (rope->layout == RKV_ROPE_HALF) return launch_rope_half<true>(a, L, stream);
+  return launch_ring_rope(a, L, vb, stream);
+}
+
+// Argument checks of one standalone tensor (rope3d_apply's rules).
+static rkv_status check_rope_tensor(const rkv_rope_tensor& t, int32_t H, const rkv_rope3d* rope) {
+  if (t.L < 0) return fail(RKV_ERR_INVALID_ARG, "L must be >= 0");
+  if (t.L == 0) return RKV_OK;
+  if (!t.x || !t.y) return fail(RKV_ERR_INVALID_ARG, "x/y is NULL");
+  const int64_t row_elems = int64_t(H) * 128;
+  if (t.x_row_stride < row_elems || t.y_row_stride < row_elems) return fail(RKV_ERR_INVALID_ARG, "row stride < H*D");
+  if (!aligned16(t.x) || !aligned16(t.y) || (t.x_row_stride * 2) % 16 || (t.y_row_stride * 2) % 16)
+    return fail(RKV_ERR_INVALID_ARG, "rows must be 16-byte aligned");
+  const uint64_t xb = uint64_t((t.L - 1) * t.x_row_stride + row_elems) * 2;
+  const uint64_t yb = uint64_t((t.L - 1) * t.y_row_stride + row_elems) * 2;
+  if (t.x != t.y && overlaps(t.x, xb, t.y, yb)) return fail(RKV_ERR_INVALID_ARG, "x and y overlap without being identical");
+  if (t.x == t.y && t.x_row_stride != t.y_row_stride) return fail(RKV_ERR_INVALID_ARG, "in-place call needs equal strides");
+  if (t.L >= (int64_t(1) << 31) || uint64_t(t.L) * H * 16 >= (uint64_t(1) << 31))
+    return fail(RKV_ERR_UNSUPPORTED, "too many rows for one launch");
+  const int64_t last_t = int64_t(t.t0) + (t.L - 1) / (int64_t(rope->grid_h) * rope->grid_w);
+  if (last_t > INT32_MAX) return fail(RKV_ERR_INVALID_ARG, "time index overflows int32");
+  return RKV_OK;
+}
+
+// rope3d_apply / rope3d_apply_batch: check, then one launch (adjacent layout)
+// or one launch per tensor (rotate-half layout).
+static rkv_status rope_batch(const rkv_rope_tensor* t, int32_t n, int32_t H, int32_t D, const rkv_rope3d* rope,
+                             cudaStream_t stream) {
+  if (D != 128) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", D);
+  rkv_status st = check_rope(rope, D);
+  if (st != RKV_OK) return st;
+  if (H < 1) return fail(RKV_ERR_INVALID_ARG, "H must be >= 1");
+  RopeRows rows[kRopeBatchMax];
+  int64_t L[kRopeBatchMax];
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    if ((st = check_rope_tensor(t[i], H, rope)) != RKV_OK) return st;
+    if (t[i].L == 0) continue;
+    const int64_t row_elems = int64_t(H) * 128;
+    const uint64_t yb = uint64_t((t[i].L - 1) * t[i].y_row_stride + row_elems) * 2;
+    for (int j = 0; j < n; ++j) {
+      if (j == i || t[j].L == 0) continue;
+      const uint64_t xb = uint64_t((t[j].L - 1) * t[j].x_row_stride + row_elems) * 2;
+      const uint64_t yb2 = uint64_t((t[j].L - 1) * t[j].y_row_stride + row_elems) * 2;
+      if (overlaps(t[i].y, yb, t[j].x, xb) || overlaps(t[i].y, yb, t[j].y, yb2))
+        return fail(RKV_ERR_INVALID_ARG, "tensor %d's output overlaps tensor %d", i, j);
+    }
+    rows[m] = RopeRows{static_cast<const uint8_t*>(t[i].x), static_cast<uint8_t*>(t[i].y), t[i].x_row_stride * 2,
+                       t[i].y_row_stride * 2, t[i].t0};
+    L[m] = t[i].L;
+    ++m;
+  }
+  if (m == 0) return RKV_OK;
+  if (rope->layout == RKV_ROPE_HALF) {
+    for (int i = 0; i < m; ++i) {
+      RopeArgs a{};
+      a.x = rows[i].x;
+      a.y = rows[i].y;
+      a.x_stride_bytes = rows[i].xs;
+      a.y_stride_bytes = rows[i].ys;
+      fill_rope_args(a, L[i], H, rows[i].t0, rope);
+      if ((st = launch_rope_half<false>(a, L[i], stream)) != RKV_OK) return st;
+    }
+    return RKV_OK;
+  }
+  RopeArgs a{};
+  fill_rope_args(a, 1, H, 0, rope);
+  return launch_rope_adj(a, rows, L, m, stream);
 }
 
 }  // namespace rkv
@@ -698,31 +806,17 @@ extern "C" rkv_status rope3d_apply(const void* x, void* y, int64_t L, int32_t H,
                                    int64_t y_row_stride, int32_t t0, const rkv_rope3d* rope, void* stream) {
   NvtxRange nvtx_range("rope3d_apply");
   clear_error();
-  if (D != 128) return fail(RKV_ERR_INVALID_ARG, "head_dim D must be 128 (got %d)", D);
-  rkv_status st = check_rope(rope, D);
-  if (st != RKV_OK) return st;
-  if (L < 0 || H < 1) return fail(RKV_ERR_INVALID_ARG, "L must be >= 0 and H >= 1");
-  if (L == 0) return RKV_OK;
-  if (!x || !y) return fail(RKV_ERR_INVALID_ARG, "x/y is NULL");
-  const int64_t row_elems = int64_t(H) * D;
-  if (x_row_stride < row_elems || y_row_stride < row_elems) return fail(RKV_ERR_INVALID_ARG, "row stride < H*D");
-  if (!aligned16(x) || !aligned16(y) || (x_row_stride * 2) % 16 || (y_row_stride * 2) % 16)
-    return fail(RKV_ERR_INVALID_ARG, "rows must be 16-byte aligned");
-  const uint64_t xb = uint64_t((L - 1) * x_row_stride + row_elems) * 2;
-  const uint64_t yb = uint64_t((L - 1) * y_row_stride + row_elems) * 2;
-  if (x != y && overlaps(x, xb, y, yb)) return fail(RKV_ERR_INVALID_ARG, "x and y overlap without being identical");
-  if (x == y && x_row_stride != y_row_stride) return fail(RKV_ERR_INVALID_ARG, "in-place call needs equal strides");
-  if (L >= (int64_t(1) << 31) || uint64_t(L) * H * 16 >= (uint64_t(1) << 31))
-    return fail(RKV_ERR_UNSUPPORTED, "too many rows for one launch");
-  const int64_t last_t = int64_t(t0) + (L - 1) / (int64_t(rope->grid_h) * rope->grid_w);
-  if (last_t > INT32_MAX) return fail(RKV_ERR_INVALID_ARG, "time index overflows int32");
+  const rkv_rope_tensor t = {x, y, L, x_row_stride, y_row_stride, t0};
+  return rope_batch(&t, 1, H, D, rope, static_cast<cudaStream_t>(stream));
+}
 
-  RopeArgs a{};
-  a.x = static_cast<const uint8_t*>(x);
-  a.y = static_cast<uint8_t*>(y);
-  a.x_stride_bytes = x_row_stride * 2;
-  a.y_stride_bytes = y_row_stride * 2;
-  return launch_rope<false>(a, L, H, t0, rope, nullptr, static_cast<cudaStream_t>(stream));
+extern "C" rkv_status rope3d_apply_batch(const rkv_rope_tensor* tensors, int32_t n, int32_t H, int32_t D,
+                                         const rkv_rope3d* rope, void* stream) {
+  NvtxRange nvtx_range("rope3d_apply_batch");
+  clear_error();
+  if (n < 0 || n > kRopeBatchMax) return fail(RKV_ERR_INVALID_ARG, "n must be in [0, %d]", kRopeBatchMax);
+  if (n > 0 && !tensors) return fail(RKV_ERR_INVALID_ARG, "tensors is NULL");
+  return rope_batch(tensors, n, H, D, rope, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new, const void* v_new,
@@ -756,8 +850,8 @@ extern "C" rkv_status kvcache_ring_update_rope(rkv_ring* ring, const void* k_new
     if (st != RKV_OK) return st;
     st = ring_timeout_flag(&vb.timeout_flag);
     if (st != RKV_OK) return st;
-    st = launch_rope<true>(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope, &vb,
-                           static_cast<cudaStream_t>(stream));
+    st = launch_ring(a, int64_t(n_frames) * ring->tokens_per_frame, ring->H, t0, rope, vb,
+                     static_cast<cudaStream_t>(stream));
     if (st != RKV_OK) return st;
   }
   ring_advance(ring, n_frames, n_evicted);

@@ -35,6 +35,12 @@ class rkv_rope3d(ctypes.Structure):
 
 
 RKV_ROPE_ADJACENT, RKV_ROPE_HALF = 0, 1
+RKV_ROPE_BATCH_MAX = 8
+
+
+class rkv_rope_tensor(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("L", ctypes.c_int64),
+                ("x_row_stride", ctypes.c_int64), ("y_row_stride", ctypes.c_int64), ("t0", ctypes.c_int32)]
 
 
 class rkv_attn_seq(ctypes.Structure):
@@ -67,6 +73,9 @@ _c = ctypes
 _lib.rope3d_apply.restype = _c.c_int
 _lib.rope3d_apply.argtypes = [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int32, _c.c_int32, _c.c_int64, _c.c_int64,
                               _c.c_int32, _c.POINTER(rkv_rope3d), _c.c_void_p]
+_lib.rope3d_apply_batch.restype = _c.c_int
+_lib.rope3d_apply_batch.argtypes = [_c.POINTER(rkv_rope_tensor), _c.c_int32, _c.c_int32, _c.c_int32,
+                                    _c.POINTER(rkv_rope3d), _c.c_void_p]
 _lib.attn_fwd_varlen_workspace_size.restype = _c.c_size_t
 _lib.attn_fwd_varlen_workspace_size.argtypes = [_c.POINTER(rkv_attn_seq), _c.c_int32, _c.c_int32, _c.c_int32]
 _lib.attn_fwd_varlen.restype = _c.c_int
@@ -168,6 +177,30 @@ def rope3d_apply(x, y=None, t0=0, rope=None, stream=None):
     _check(_lib.rope3d_apply(x.data_ptr(), y.data_ptr(), L, H, D, xs, ys, int(t0), ctypes.byref(rope),
                              _stream(stream)))
     return y
+
+
+def rope3d_apply_batch(items, rope=None, stream=None):
+    """rope3d_apply on several tensors in one launch.  items: sequence of
+    (x, y, t0) with x, y bf16 [L, H, 128] CUDA tensors of the same H (y=None ->
+    new tensor, y=x -> in place).  Returns the list of y."""
+    import torch
+    outs = []
+    arr = (rkv_rope_tensor * max(1, len(items)))()
+    H = None
+    for i, (x, y, t0) in enumerate(items):
+        if y is None:
+            y = torch.empty_like(x)
+        xs, ys = _rows(x, "x"), _rows(y, "y")
+        if tuple(x.shape) != tuple(y.shape):
+            raise ValueError("x and y shapes differ")
+        if H is None:
+            H = x.shape[1]
+        elif x.shape[1] != H:
+            raise ValueError("all tensors of a batch must have the same number of heads")
+        arr[i] = rkv_rope_tensor(x.data_ptr(), y.data_ptr(), x.shape[0], xs, ys, int(t0))
+        outs.append(y)
+    _check(_lib.rope3d_apply_batch(arr, len(items), H or 1, 128, ctypes.byref(rope), _stream(stream)))
+    return outs
 
 
 class AttnSeq:

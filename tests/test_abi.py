@@ -200,6 +200,37 @@ def test_make_rope_variants(rkv):
         rkv.make_rope(4, 6, layout="interleaved")
 
 
+def _batch(rkv, items):
+    arr = (rkv.rkv_rope_tensor * max(1, len(items)))()
+    for i, (x, y, L, t0) in enumerate(items):
+        arr[i] = rkv.rkv_rope_tensor(x, y, L, 256, 256, t0)
+    return arr
+
+
+def test_rope_batch_rejects(rkv):
+    lib = rkv.lib()
+    r = rope(rkv)
+    ok = [(0x1000, 0x90000000, 72, 0), (0x200000, 0xA0000000, 120, 1)]
+    # more tensors than a launch takes
+    arr = _batch(rkv, ok * 5)
+    assert lib.rope3d_apply_batch(arr, 9, 2, 128, ctypes.byref(r), None) == rkv.RKV_ERR_INVALID_ARG
+    assert "n must be" in rkv.rkv_last_error_string()
+    assert lib.rope3d_apply_batch(None, 2, 2, 128, ctypes.byref(r), None) == rkv.RKV_ERR_INVALID_ARG
+    # one tensor's output over another's input or output
+    for bad in ([(0x1000, 0x90000000, 72, 0), (0x200000, 0x90000100, 120, 1)],
+                [(0x1000, 0x90000000, 72, 0), (0x90000100, 0xA0000000, 120, 1)]):
+        assert lib.rope3d_apply_batch(_batch(rkv, bad), 2, 2, 128, ctypes.byref(r), None) == rkv.RKV_ERR_INVALID_ARG
+        assert "overlaps tensor" in rkv.rkv_last_error_string()
+    # a tensor's own rules still apply
+    bad = [(0x1000, 0x90000000, 72, 0), (0x0, 0xA0000000, 120, 1)]
+    assert lib.rope3d_apply_batch(_batch(rkv, bad), 2, 2, 128, ctypes.byref(r), None) == rkv.RKV_ERR_INVALID_ARG
+    assert "NULL" in rkv.rkv_last_error_string()
+    # nothing to do: no tensors, or only empty ones
+    assert lib.rope3d_apply_batch(None, 0, 2, 128, ctypes.byref(r), None) == rkv.RKV_OK
+    empty = [(0x0, 0x0, 0, 0), (0x0, 0x0, 0, 3)]
+    assert lib.rope3d_apply_batch(_batch(rkv, empty), 2, 2, 128, ctypes.byref(r), None) == rkv.RKV_OK
+
+
 def test_rope_zero_rows_is_a_noop(rkv):
     r = rope(rkv)
     assert rkv.lib().rope3d_apply(None, None, 0, 2, 128, 256, 256, 0, ctypes.byref(r), None) == rkv.RKV_OK

@@ -80,3 +80,58 @@ def test_chunk_on_three_axes():
 
 def test_large_time_index():
     check_rope(200, 2, 4, 6, 1000, 18)
+
+
+def _bits(t):
+    return to_bits(t)
+
+
+def test_batch_matches_separate_calls_and_oracle():
+    # Q and K of the mid-size pass in one launch, plus a ragged third tensor
+    # rotated in place: each output bit-identical to its own rope3d_apply and
+    # within one ulp of the oracle
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    H, D = MID.heads, 128
+    rope = rkv.make_rope(MID.grid_h, MID.grid_w)
+    shapes = [(MID.Lq, MID.q_t0, 31), (MID.Lk, MID.k_t0, 32), (1000, 4, 33)]
+    xs = [bf16_normal_bits(seed, (L, H, D)) for L, _, seed in shapes]
+    devs = [to_dev(x) for x in xs]
+    inplace = devs[2].clone()
+    outs = rkv.rope3d_apply_batch([(devs[0], None, shapes[0][1]), (devs[1], None, shapes[1][1]),
+                                   (inplace, inplace, shapes[2][1])], rope=rope)
+    for i, (L, t0, _) in enumerate(shapes):
+        alone = rkv.rope3d_apply(devs[i], t0=t0, rope=rope)
+        torch.cuda.synchronize()
+        assert np.array_equal(_bits(outs[i]), _bits(alone)), i
+        ref = f64_to_bf16_bits(rope3d_ref(bf16_bits_to_f64(xs[i]), t0, MID.grid_h, MID.grid_w))
+        assert int(bf16_ulp_distance(_bits(outs[i]), ref).max()) <= 1, i
+
+
+def test_batch_full_size_q_and_k():
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    H, D = DENOISE.heads, 128
+    rope = rkv.make_rope(DENOISE.grid_h, DENOISE.grid_w)
+    q = to_dev(bf16_normal_bits(DENOISE.seed, (DENOISE.Lq, H, D)))
+    k = to_dev(bf16_normal_bits(DENOISE.seed + 1, (DENOISE.Lk, H, D)))
+    yq, yk = rkv.rope3d_apply_batch([(q, None, DENOISE.q_t0), (k, None, DENOISE.k_t0)], rope=rope)
+    aq = rkv.rope3d_apply(q, t0=DENOISE.q_t0, rope=rope)
+    ak = rkv.rope3d_apply(k, t0=DENOISE.k_t0, rope=rope)
+    torch.cuda.synchronize()
+    assert torch.equal(yq.view(torch.int16), aq.view(torch.int16))
+    assert torch.equal(yk.view(torch.int16), ak.view(torch.int16))
+
+
+def test_batch_strided_odd_split_and_rotate_half():
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    H, D = 2, 128
+    for rope in (rkv.make_rope(5, 7, (21, 2, 41)), rkv.make_rope(5, 7, layout="half")):
+        wide = to_dev(bf16_normal_bits(41, (300, 3 * H, D)))[:, :H, :]
+        plain = to_dev(bf16_normal_bits(42, (77, H, D)))
+        y1, y2 = rkv.rope3d_apply_batch([(wide, None, 3), (plain, None, 0)], rope=rope)
+        a1 = rkv.rope3d_apply(wide, t0=3, rope=rope)
+        a2 = rkv.rope3d_apply(plain, t0=0, rope=rope)
+        torch.cuda.synchronize()
+        assert np.array_equal(_bits(y1), _bits(a1)) and np.array_equal(_bits(y2), _bits(a2))
