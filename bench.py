@@ -689,6 +689,8 @@ def profile_case(args):
         elif case == "rope":
             rkv.rope3d_apply(t["q"], yq, t0=Q_T0, rope=rope)
             rkv.rope3d_apply(t["k"], yk, t0=K_T0, rope=rope)
+        elif case == "rope_batched":
+            rkv.rope3d_apply_batch([(t["q"], yq, Q_T0), (t["k"], yk, K_T0)], rope=rope)
         else:
             raise SystemExit(f"unknown --profile-case {case}")
 
@@ -741,7 +743,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 30-layer rolling sweep measurement")
-    ap.add_argument("--profile-case", choices=["attention", "attention_qonly", "ring", "ring_rope", "rope"],
+    ap.add_argument("--profile-case", choices=["attention", "attention_qonly", "ring", "ring_rope", "rope", "rope_batched"],
                     help="run only W + K launches of one call (for ncu); prints nothing")
     args = ap.parse_args()
     if args.impl == "reference":

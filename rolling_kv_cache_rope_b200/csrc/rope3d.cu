@@ -74,7 +74,7 @@ constexpr int rope_threads() { return kRing ? 256 : 1024; }
 constexpr int kRopeUnroll = 4;
 constexpr int kRopeBatchMax = RKV_ROPE_BATCH_MAX;   // tensors of one rope3d_apply_batch launch
 constexpr int kRopeMaxEntries = 4096;  // 64 KB of per-pair entries per CTA (rotate-half)
-constexpr int kAdjMaxEntries = 1024;   // 64 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
+constexpr int kAdjMaxEntries = 2048;   // 128 KB of chunk entries (4 float4 arrays) per CTA (adjacent)
 constexpr int kRingRopeThreads = 640;   // rotated ring insert, at most: warp 0 copies V, the rest rotate K
 constexpr int kRingRopeSmem = 227 * 1024 - 256;   // its dynamic shared memory at most (V stages + table)
 
