@@ -121,3 +121,9 @@ def test_ring_rope_rejects_grid_mismatch():
     with pytest.raises(rkv.RkvError) as e:
         rkv.kvcache_ring_update_rope(ring, k, k.clone(), 0, rkv.make_rope(5, 5), 1)
     assert e.value.status == 1 and (ring.head, ring.count) == (0, 0)
+
+
+def test_ring_rope_rows_wider_than_a_piece():
+    # 160 heads: 40 KB rows; V moves in 32 KB + 8 KB pieces, K rows are
+    # rotated 1,024 chunks at a time by each CTA's threads
+    run_ring_rope(4, 2, 3, 160, [3, 2, 4], seed=81)

@@ -135,3 +135,21 @@ def test_batch_strided_odd_split_and_rotate_half():
         a2 = rkv.rope3d_apply(plain, t0=0, rope=rope)
         torch.cuda.synchronize()
         assert np.array_equal(_bits(y1), _bits(a1)) and np.array_equal(_bits(y2), _bits(a2))
+
+
+def test_rows_of_more_chunks_than_threads():
+    # 160 heads: 2,560 chunks per row against 1,024 threads per CTA
+    check_rope(40, 160, 2, 3, 1, 22)
+
+
+def test_batch_of_eight():
+    need_gpu()
+    from rolling_kv_cache_rope_b200 import rkv
+    H, D = 3, 128
+    rope = rkv.make_rope(4, 6)
+    xs = [to_dev(bf16_normal_bits(50 + i, (7 + 29 * i, H, D))) for i in range(8)]
+    outs = rkv.rope3d_apply_batch([(x, None, i) for i, x in enumerate(xs)], rope=rope)
+    for i, x in enumerate(xs):
+        alone = rkv.rope3d_apply(x, t0=i, rope=rope)
+        torch.cuda.synchronize()
+        assert np.array_equal(_bits(outs[i]), _bits(alone)), i
